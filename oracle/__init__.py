@@ -1,0 +1,132 @@
+"""fp64 CPU oracle for block-causal attention forward + JVP (test infrastructure).
+
+Only the tests, the package's smoke check and the benchmark's CPU-baseline arm
+import this package. The product path never does. The arithmetic lives in
+`oracle.c` (plain C, fp64, OpenMP over rows); this module only compiles it with
+gcc and marshals arrays through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_F64, _F32, _BF16 = 0, 1, 2
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+                        "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i64, i32, dbl, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
+        lib.oracle_visible.argtypes = [i64, i64, i64, i32, i64, i64]
+        lib.oracle_visible.restype = i32
+        lib.oracle_visible_pairs.argtypes = [i64, i64, i64, i32]
+        lib.oracle_visible_pairs.restype = i64
+        lib.oracle_attn_fwd_jvp_rows.argtypes = [vp] * 6 + [i32, i64, i64, i64, dbl,
+                                                            i64, i64, i64, i32, vp, i64,
+                                                            vp, vp, vp, vp, i32]
+        lib.oracle_attn_fwd_jvp_rows.restype = i32
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = i32
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return _load().oracle_max_threads()
+
+
+def visible(mask, qi: int, kj: int) -> bool:
+    """Whether query token qi may attend to key token kj under `mask`
+    (a MaskDesc or a (T, c, F, tf) tuple)."""
+    T, c, F, tf = _mask_tuple(mask)
+    return bool(_load().oracle_visible(T, c, F, tf, qi, kj))
+
+
+def visible_pairs(mask) -> int:
+    """Visible (query, key) pairs of one head, counted by brute force."""
+    T, c, F, tf = _mask_tuple(mask)
+    return int(_load().oracle_visible_pairs(T, c, F, tf))
+
+
+def _mask_tuple(mask):
+    if hasattr(mask, "as_tuple"):
+        return mask.as_tuple()
+    return tuple(int(x) for x in mask)
+
+
+def _as_host(t: torch.Tensor):
+    t = t.detach()
+    if t.device.type != "cpu":
+        t = t.cpu()
+    t = t.contiguous()
+    if t.dtype == torch.float64:
+        return t, _F64
+    if t.dtype == torch.float32:
+        return t, _F32
+    if t.dtype == torch.bfloat16:
+        return t, _BF16
+    raise TypeError(f"oracle: unsupported dtype {t.dtype}")
+
+
+def attn_fwd_jvp_rows(q, k, v, tq, tk, tv, mask, scale=None, rows=None, nthreads=0):
+    """fp64 O, tO, LSE, tLSE for selected rows.
+
+    q..tv: [B, H, N, D] tensors of one dtype (fp64, fp32 or bf16; values are
+    widened to double exactly). rows: flat ids bh*N + i (default: all rows).
+    Returns numpy arrays o [R, D], to [R, D], lse [R], tlse [R] (float64).
+    """
+    ts = [_as_host(t) for t in (q, k, v, tq, tk, tv)]
+    dtypes = {d for _, d in ts}
+    if len(dtypes) != 1:
+        raise TypeError("oracle: all six inputs must share one dtype")
+    dtype = dtypes.pop()
+    B, H, N, D = q.shape
+    for t, _ in ts:
+        if tuple(t.shape) != (B, H, N, D):
+            raise ValueError("oracle: shape mismatch")
+    T, c, F, tf = _mask_tuple(mask)
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(D))
+    if rows is None:
+        rows = torch.arange(B * H * N, dtype=torch.int64)
+    rows = torch.as_tensor(rows, dtype=torch.int64).contiguous()
+    R = rows.numel()
+    o = np.zeros((R, D), np.float64)
+    to = np.zeros((R, D), np.float64)
+    lse = np.zeros((R,), np.float64)
+    tlse = np.zeros((R,), np.float64)
+    rc = _load().oracle_attn_fwd_jvp_rows(
+        *[t.data_ptr() for t, _ in ts], dtype, B * H, N, D, float(scale),
+        T, c, F, tf, rows.data_ptr(), R,
+        o.ctypes.data, to.ctypes.data, lse.ctypes.data, tlse.ctypes.data, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle: rejected arguments")
+    return o, to, lse, tlse
+
+
+def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale=None, nthreads=0):
+    """Full outputs shaped like the inputs: o, to [B, H, N, D]; lse, tlse [B, H, N]."""
+    B, H, N, D = q.shape
+    o, to, lse, tlse = attn_fwd_jvp_rows(q, k, v, tq, tk, tv, mask, scale, None, nthreads)
+    return (o.reshape(B, H, N, D), to.reshape(B, H, N, D),
+            lse.reshape(B, H, N), tlse.reshape(B, H, N))
