@@ -1,0 +1,325 @@
+"""Benchmark: block-causal attention forward + JVP on B200.
+
+One step = one call of the fused kernel over the whole workload (every head of
+every batch entry), inputs resident in HBM. Default workload: the teacher-forcing
+frame-wise Wan2.1-1.3B-shaped layout (B=1, H=12, D=128, 21 clean + 21 noisy
+latent frames of 1560 tokens, N=65520, bf16 in / fp32 accumulate).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line on rank 0. Multi-GPU runs (torchrun) give every rank its
+own copy of the workload (independent problems, no data-path collective) and
+report whole-job throughput over the slowest rank.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from masked_attention_jvp_b200.workloads import WORKLOADS, BENCH_WORKLOAD, make_inputs  # noqa: E402
+
+METRIC = "block-causal attention fwd+JVP TFLOP/s and % of B200 dense BF16 peak"
+DENSE_BF16_SPEC_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w, extra=None):
+    m = w.mask
+    cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
+           "tokens_per_frame": m.tokens_per_frame, "frames_per_chunk": m.frames_per_chunk,
+           "n_frames": m.n_frames, "tf_layout": m.tf_layout,
+           "dtype_in": str(w.dtype).split(".")[-1], "accumulate": "fp32",
+           "l2": "inputs larger than L2 (6 bf16 tensors of %.2f GB total per step)" % (
+               6 * w.B * w.H * w.N * w.D * 2 / 1e9)}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def flops_of(w):
+    from masked_attention_jvp_b200 import flops
+    return flops(w.B, w.H, w.D, w.mask)
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_rows_flops(w, rows):
+    """12 D flops per visible key of each sampled row (same count as the GPU)."""
+    import oracle
+    m = w.mask
+    G, L = m.frames_per_chunk * m.tokens_per_frame, m.n_frames * m.tokens_per_frame
+    total = 0
+    for r in rows.tolist():
+        i = r % w.N
+        if not m.tf_layout or i < L:
+            nk = (i // G + 1) * G
+        else:
+            nk = ((i - L) // G) * G + G
+        total += nk
+    return 12 * w.D * total
+
+
+def time_oracle(w, target_s=15.0, host_inputs=None):
+    """Times the oracle as it stands on a bounded row sample of workload `w`.
+    Returns (TFLOP/s, seconds, rows, threads, description)."""
+    import oracle
+    from masked_attention_jvp_b200.workloads import sample_rows
+    ins = host_inputs if host_inputs is not None else make_inputs(w, "cpu")
+    threads = oracle.max_threads()
+    per_head = 4
+    rows = sample_rows(w, per_head, seed_offset=77)
+    t0 = time.perf_counter()
+    oracle.attn_fwd_jvp_rows(*ins, w.mask, scale=w.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    # scale the sample to about target_s seconds of CPU work
+    per_head = max(1, min(w.N, int(per_head * target_s / max(dt, 1e-3))))
+    rows = sample_rows(w, per_head, seed_offset=78)
+    t0 = time.perf_counter()
+    oracle.attn_fwd_jvp_rows(*ins, w.mask, scale=w.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    fl = oracle_rows_flops(w, rows)
+    desc = (f"{rows.numel()} seeded query rows ({per_head} per head x {w.B * w.H} heads) of "
+            f"{w.name}, fp64 oracle, {threads} OpenMP threads")
+    return fl / dt / 1e12, dt, rows.numel(), threads, desc
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def bench_gpu(args, rank, world, local_rank):
+    import masked_attention_jvp_b200 as caj
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    host = make_inputs(w, "cpu")
+    ins = [t.to(dev) for t in host]
+    o = torch.empty_like(ins[0])
+    to = torch.empty_like(ins[0])
+    lse = torch.empty(ins[0].shape[:3], dtype=torch.float32, device=dev)
+    tlse = torch.empty_like(lse)
+    stream = torch.cuda.current_stream(dev)
+    fl = flops_of(w)
+
+    def step():
+        caj.attn_fwd_jvp_out(*ins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    caj.device_status()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    caj.device_status()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * fl * args.steps / (total_ms / 1e3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    pinned = [t.pin_memory() for t in host]
+    h2d = sum(t.numel() * t.element_size() for t in pinned)
+    d2h = 2 * o.numel() * o.element_size() + 2 * lse.numel() * 4
+    e2e_steps = max(1, min(args.steps, 5))
+    caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)  # warm the host path once
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * fl * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    if rank != 0:
+        return None
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    kernel_ms = statistics.mean(per)
+    achieved = fl / (kernel_ms / 1e3) / 1e12
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q,k,v; N(0,0.5^2) tangents)",
+        "config": workload_config(w, {"parallelism": f"replica x{world}" if world > 1 else "single GPU"}),
+        "pct_of_dense_bf16_peak": round(100.0 * value / world / DENSE_BF16_SPEC_TFLOPS, 2),
+        "ms_per_step_min": round(min(per), 4), "ms_per_step_median": round(statistics.median(per), 4),
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16 burst (cuBLAS)", "kernel": "fwd_jvp_sm100_kernel<128>"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tf, dt, nrows, threads, desc = time_oracle(w, host_inputs=host)
+        line["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+    return line
+
+
+def bench_reference(args, rank):
+    """The oracle as it stands, on the host cores: each step a bounded row sample."""
+    if rank != 0:
+        return None
+    import oracle
+    from masked_attention_jvp_b200.workloads import sample_rows
+    w = WORKLOADS[args.workload]
+    host = make_inputs(w, "cpu")
+    threads = oracle.max_threads()
+    per_head = 8
+    rows_list = [sample_rows(w, per_head, seed_offset=200 + i) for i in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        oracle.attn_fwd_jvp_rows(*host, w.mask, scale=w.scale, rows=rows_list[i])
+    fl = 0
+    t0 = time.perf_counter()
+    for i in range(args.warmup, args.warmup + args.steps):
+        oracle.attn_fwd_jvp_rows(*host, w.mask, scale=w.scale, rows=rows_list[i])
+        fl += oracle_rows_flops(w, rows_list[i])
+    dt = time.perf_counter() - t0
+    value = fl / dt / 1e12
+    desc = (f"per step {per_head} seeded query rows per head x {w.B * w.H} heads of {w.name}, "
+            f"fp64 oracle, {threads} OpenMP threads")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": workload_config(w),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = bench_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = bench_gpu(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,135 @@
+/*
+ * libcausaljvp -- fused forward + forward-mode JVP of block-causal softmax
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the masked FlashAttention JVP of the Causal-rCM paper
+ * (arXiv 2606.25473), appendix B "FlashAttention-2 JVP kernel with custom
+ * mask", eq. 42-45 and Algorithm 1. Per (batch, head), with S = scale*Q K^T + M,
+ * P = softmax(S), O = P V:
+ *   tS   = scale * (tQ K^T + Q tK^T)                          (eq. 43)
+ *   tO   = (P o (tS - rowsum(P o tS))) V + P tV               (eq. 44)
+ *   LSE  = log sum_j exp(S_ij)         (natural log)
+ *   tLSE = rowsum(P o tS)
+ * M is 0 where a query may attend to a key and -inf elsewhere; it carries no
+ * tangent (appendix B, text after eq. 43). The mask family is the block-causal
+ * one of section 3.1.1 (teacher forcing, eq. 8) and section 4 (frame-wise c1-1
+ * and chunk-wise c3-3 chunking), described by caj_mask_desc below.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named q, k, v, tq, tk, tv, o, to, lse, tlse are DEVICE pointers on
+ *    the current CUDA device. The caller owns and allocates every buffer; the
+ *    library allocates no device memory per call.
+ *  - Tensors q..tv, o, to are [B, H, N, D] contiguous (D fastest), 16-byte
+ *    aligned. lse and tlse are [B, H, N] fp32, 4-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls are asynchronous on that stream; nothing synchronises implicitly.
+ *  - Argument errors are detected on the host, before anything is launched, and
+ *    leave the outputs untouched.
+ */
+#ifndef CAUSALJVP_H
+#define CAUSALJVP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CAJ_OK = 0,
+  CAJ_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad shape or mask descriptor */
+  CAJ_ERR_UNSUPPORTED = 2,    /* valid request this build does not implement (e.g. D=96) */
+  CAJ_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed; see caj_last_cuda_error */
+  CAJ_ERR_DEVICE_TIMEOUT = 4  /* a kernel gave up on a bounded wait (reported asynchronously) */
+} caj_status;
+
+typedef enum { CAJ_DTYPE_F32 = 0, CAJ_DTYPE_BF16 = 1 } caj_dtype;
+
+/*
+ * Block-causal mask (Causal-rCM section 3.1.1 and section 4). Tokens come in
+ * frames of `tokens_per_frame` (T) tokens and frames in chunks of
+ * `frames_per_chunk` (c) frames; G = c*T tokens per chunk, L = n_frames*T.
+ *   tf_layout = 0: N = L. Query i sees every key of its own chunk and of all
+ *                  earlier chunks (diffusion-forcing / inference layout).
+ *   tf_layout = 1: N = 2L, packed [clean | noisy] (teacher forcing, eq. 8).
+ *                  A clean query of chunk j sees clean chunks <= j. A noisy
+ *                  query of chunk j sees clean chunks < j and its own noisy
+ *                  chunk j. Clean queries see no noisy key.
+ * Requirements: all fields > 0 (tf_layout in {0,1}), n_frames % frames_per_chunk == 0.
+ */
+typedef struct {
+  int32_t tokens_per_frame;
+  int32_t frames_per_chunk;
+  int32_t n_frames;
+  int32_t tf_layout;
+} caj_mask_desc;
+
+/* Problem shape. dtype is a caj_dtype and applies to q..tv, o and to.
+ * scale <= 0 selects 1/sqrt(D). */
+typedef struct {
+  int32_t B, H, N, D;
+  int32_t dtype;
+  float scale;
+} caj_problem;
+
+/*
+ * Forward + JVP of block-causal attention (appendix B eq. 42-45, Algorithm 1).
+ *   in : q, k, v, tq, tk, tv   [B,H,N,D] of prob->dtype, read only
+ *   out: o, to                 [B,H,N,D] of prob->dtype, fully overwritten
+ *        lse, tlse             [B,H,N] fp32, fully overwritten
+ * Supported: D in {64, 128}; dtype BF16 (tensor-core path, fp32 accumulation)
+ * or F32 (CUDA-core fp32 path); N == n_frames*tokens_per_frame*(tf_layout?2:1);
+ * B*H <= 65535; N <= 1048576.
+ * Returns CAJ_OK once the kernel is enqueued, CAJ_ERR_INVALID_ARG /
+ * CAJ_ERR_UNSUPPORTED without launching, or CAJ_ERR_CUDA if the launch failed.
+ * Device-side bounded-wait failures are reported by caj_last_device_status.
+ */
+caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v,
+                            const void *tq, const void *tk, const void *tv,
+                            const caj_problem *prob, const caj_mask_desc *mask,
+                            void *o, void *to, float *lse, float *tlse,
+                            void *stream);
+
+/* Synchronises `stream`, then reads and clears the library's device error word.
+ * Returns CAJ_OK, CAJ_ERR_DEVICE_TIMEOUT (a kernel abandoned a wait; its
+ * outputs are undefined) or CAJ_ERR_CUDA. */
+caj_status caj_last_device_status(void *stream);
+
+/* Detail of the last device error: which wait gave up (0 if none). Valid after
+ * caj_last_device_status returned CAJ_ERR_DEVICE_TIMEOUT. */
+uint32_t caj_last_device_error_code(void);
+
+/* Human-readable name of a status. Never NULL. */
+const char *caj_status_string(caj_status s);
+
+/* Text of the last CUDA error seen by this library on this thread ("" if none). */
+const char *caj_last_cuda_error(void);
+
+/* ---- host-side mask and schedule queries (no GPU needed) ---- */
+
+/* Checks a mask descriptor against N. Returns CAJ_OK or CAJ_ERR_INVALID_ARG. */
+caj_status caj_validate_mask(const caj_mask_desc *mask, int32_t N);
+
+/* Visible (query, key) pairs of one head, in closed form; -1 on a bad mask.
+ * Work of one call is 12 * D * visible_pairs * B * H floating-point operations. */
+int64_t caj_visible_pairs(const caj_mask_desc *mask);
+
+/* Keys that query row `row` may attend to, as up to two half-open intervals
+ * [r[0], r[1]) and [r[2], r[3]) (an empty interval has r[2] == r[3]).
+ * Returns CAJ_OK or CAJ_ERR_INVALID_ARG. */
+caj_status caj_row_key_ranges(const caj_mask_desc *mask, int32_t row, int32_t r[4]);
+
+/* The key tiles of width `block_n` the kernel visits for the query tile
+ * [q0, q1): up to two half-open tile-index ranges [t[0], t[1]) and [t[2], t[3]),
+ * ascending and disjoint. Returns the number of tiles, or -1 on a bad argument. */
+int32_t caj_qtile_key_tiles(const caj_mask_desc *mask, int32_t q0, int32_t q1,
+                            int32_t block_n, int32_t t[4]);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t caj_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CAUSALJVP_H */

@@ -1,0 +1,129 @@
+"""Fused forward + forward-mode JVP of block-causal softmax attention on B200.
+
+Public API (a thin layer over the C-ABI library libcausaljvp):
+
+    o, to, lse, tlse = attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale=None)
+
+q..tv are [B, H, N, D] tensors (bf16 for the tensor-core path, fp32 for the
+CUDA-core fp32 path), `mask` a MaskDesc (or a (tokens_per_frame,
+frames_per_chunk, n_frames, tf_layout) tuple). With CUDA tensors everything
+stays on the device and the call is asynchronous on the current stream. With
+CPU tensors the inputs are copied to the current CUDA device and the outputs
+copied back (the end-to-end path).
+
+The operation is the masked FlashAttention JVP of the Causal-rCM paper
+(appendix B, eq. 42-45): O = softmax(scale Q K^T + M) V,
+tO = (P o (tS - rowsum(P o tS))) V + P tV with tS = scale (tQ K^T + Q tK^T),
+LSE (natural log) and tLSE = rowsum(P o tS).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import CajError, EXPORTED, LIB_PATH
+from .workloads import MaskDesc
+
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "MaskDesc", "CajError", "visible_pairs",
+           "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
+           "BLOCK_M", "BLOCK_N"]
+
+BLOCK_M = 128  # query rows per tile of both kernels
+BLOCK_N = 64   # keys per tile of the tensor-core kernel
+
+_DTYPES = {torch.float32: _lib.CAJ_DTYPE_F32, torch.bfloat16: _lib.CAJ_DTYPE_BF16}
+
+
+def visible_pairs(mask) -> int:
+    """Visible (query, key) pairs of one head (closed form, from the library)."""
+    n = _lib.lib().caj_visible_pairs(ctypes.byref(_lib.mask_c(mask)))
+    if n < 0:
+        raise ValueError(f"invalid mask descriptor {mask}")
+    return int(n)
+
+
+def flops(B: int, H: int, D: int, mask) -> int:
+    """Algorithmic floating-point work of one call: 12 D per visible pair per head
+    (six products of 2 D flops: S, two for tS, O, two for tO)."""
+    return 12 * D * visible_pairs(mask) * B * H
+
+
+def row_key_ranges(mask, row: int):
+    r = (ctypes.c_int32 * 4)()
+    _lib.check(_lib.lib().caj_row_key_ranges(ctypes.byref(_lib.mask_c(mask)), int(row), r),
+               "caj_row_key_ranges")
+    return (r[0], r[1]), (r[2], r[3])
+
+
+def qtile_key_tiles(mask, q0: int, q1: int, block_n: int = BLOCK_N):
+    t = (ctypes.c_int32 * 4)()
+    n = _lib.lib().caj_qtile_key_tiles(ctypes.byref(_lib.mask_c(mask)), int(q0), int(q1),
+                                       int(block_n), t)
+    if n < 0:
+        raise ValueError("caj_qtile_key_tiles rejected its arguments")
+    return n, (t[0], t[1]), (t[2], t[3])
+
+
+def device_status(stream: Optional[torch.cuda.Stream] = None):
+    """Synchronise the stream and raise CajError if a kernel gave up on a wait."""
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    _lib.check(_lib.lib().caj_last_device_status(ctypes.c_void_p(s)), "caj_last_device_status")
+
+
+def _problem(q: torch.Tensor, scale: Optional[float]) -> _lib.ProblemC:
+    B, H, N, D = q.shape
+    return _lib.ProblemC(B, H, N, D, _DTYPES[q.dtype], float(scale) if scale else 0.0)
+
+
+def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optional[float] = None,
+                     stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Writes into caller-provided CUDA tensors o, to [B,H,N,D] and lse, tlse [B,H,N] fp32."""
+    ins = (q, k, v, tq, tk, tv)
+    for t in ins + (o, to, lse, tlse):
+        if not t.is_cuda:
+            raise ValueError("attn_fwd_jvp_out: all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("attn_fwd_jvp_out: tensors must be contiguous")
+    if q.dtype not in _DTYPES or any(t.dtype != q.dtype for t in ins + (o, to)):
+        raise ValueError("attn_fwd_jvp_out: q..tv, o, to must share one dtype (bf16 or fp32)")
+    if any(t.shape != q.shape for t in ins + (o, to)):
+        raise ValueError("attn_fwd_jvp_out: shape mismatch")
+    if lse.dtype != torch.float32 or tlse.dtype != torch.float32 or lse.shape != q.shape[:3] \
+            or tlse.shape != q.shape[:3]:
+        raise ValueError("attn_fwd_jvp_out: lse/tlse must be fp32 [B,H,N]")
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    prob = _problem(q, scale)
+    st = _lib.lib().caj_attn_fwd_jvp(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
+                                     ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)),
+                                     ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(to.data_ptr()),
+                                     ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(tlse.data_ptr()),
+                                     ctypes.c_void_p(s))
+    _lib.check(st)
+
+
+def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None):
+    """Returns (o, to, lse, tlse). See the module docstring."""
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        ins = [t.to(dev, non_blocking=True) for t in (q, k, v, tq, tk, tv)]
+    else:
+        ins = [q, k, v, tq, tk, tv]
+    q_ = ins[0]
+    o = torch.empty_like(q_)
+    to = torch.empty_like(q_)
+    lse = torch.empty(q_.shape[:3], dtype=torch.float32, device=q_.device)
+    tlse = torch.empty_like(lse)
+    attn_fwd_jvp_out(*ins, mask, o, to, lse, tlse, scale=scale)
+    if host:
+        outs = []
+        for t in (o, to, lse, tlse):
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h.copy_(t, non_blocking=True)
+            outs.append(h)
+        torch.cuda.current_stream().synchronize()
+        return tuple(outs)
+    return o, to, lse, tlse

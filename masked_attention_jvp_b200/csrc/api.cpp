@@ -1,0 +1,249 @@
+// C-ABI front end of libcausaljvp: argument validation, the query-tile launch
+// order, TMA descriptor construction and kernel dispatch. See
+// include/causaljvp.h for the contract of every entry point.
+#include "causaljvp.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <memory>
+#include <mutex>
+#include <vector>
+
+#include "kernels.h"
+#include "mask_schedule.h"
+
+namespace {
+
+thread_local char g_cuda_msg[256] = "";
+uint32_t g_last_device_code = 0;
+
+caj_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_cuda_msg, sizeof g_cuda_msg, "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return CAJ_ERR_CUDA;
+}
+
+bool geom_from_desc(const caj_mask_desc *m, caj::MaskGeom *g) {
+  if (!m) return false;
+  const int64_t T = m->tokens_per_frame, c = m->frames_per_chunk, F = m->n_frames;
+  if (T <= 0 || c <= 0 || F <= 0) return false;
+  if (m->tf_layout != 0 && m->tf_layout != 1) return false;
+  if (F % c != 0) return false;
+  const int64_t L = F * T, N = L * (m->tf_layout ? 2 : 1);
+  if (N > (int64_t(1) << 30)) return false;
+  g->G = int32_t(c * T);
+  g->L = int32_t(L);
+  g->N = int32_t(N);
+  g->tf = m->tf_layout;
+  return true;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime so the
+// library needs no link-time dependency on libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_tiled() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over [BH, N, D] (innermost first), box = 64 columns x rows x 1,
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *base, int BH, int N, int D,
+                int box_rows) {
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(N) * D * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Per-device check that this is an sm_100 part (cached).
+caj_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  static std::mutex mu;
+  static std::vector<int> state;  // 0 unknown, 1 ok, 2 unsupported
+  std::lock_guard<std::mutex> lock(mu);
+  if (int(state.size()) <= dev) state.resize(dev + 1, 0);
+  if (state[dev] == 0) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return state[dev] == 1 ? CAJ_OK : CAJ_ERR_UNSUPPORTED;
+}
+
+uint64_t wait_timeout_ns() {
+  static uint64_t ns = [] {
+    const char *s = std::getenv("CAJ_WAIT_TIMEOUT_MS");
+    double ms = s ? std::atof(s) : 0.0;
+    if (!(ms > 0.0)) ms = 2000.0;
+    return uint64_t(ms * 1e6);
+  }();
+  return ns;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *caj_status_string(caj_status s) {
+  switch (s) {
+    case CAJ_OK: return "CAJ_OK";
+    case CAJ_ERR_INVALID_ARG: return "CAJ_ERR_INVALID_ARG";
+    case CAJ_ERR_UNSUPPORTED: return "CAJ_ERR_UNSUPPORTED";
+    case CAJ_ERR_CUDA: return "CAJ_ERR_CUDA";
+    case CAJ_ERR_DEVICE_TIMEOUT: return "CAJ_ERR_DEVICE_TIMEOUT";
+  }
+  return "CAJ_ERR_UNKNOWN";
+}
+
+const char *caj_last_cuda_error(void) { return g_cuda_msg; }
+
+int32_t caj_version(void) { return 100; }
+
+caj_status caj_validate_mask(const caj_mask_desc *mask, int32_t N) {
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g)) return CAJ_ERR_INVALID_ARG;
+  return g.N == N ? CAJ_OK : CAJ_ERR_INVALID_ARG;
+}
+
+int64_t caj_visible_pairs(const caj_mask_desc *mask) {
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g)) return -1;
+  return caj::visible_pairs(g);
+}
+
+caj_status caj_row_key_ranges(const caj_mask_desc *mask, int32_t row, int32_t r[4]) {
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g) || !r || row < 0 || row >= g.N) return CAJ_ERR_INVALID_ARG;
+  caj::row_key_ranges(g, row, r[0], r[1], r[2], r[3]);
+  return CAJ_OK;
+}
+
+int32_t caj_qtile_key_tiles(const caj_mask_desc *mask, int32_t q0, int32_t q1, int32_t block_n,
+                            int32_t t[4]) {
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g) || !t || block_n <= 0 || q0 < 0 || q1 <= q0 || q1 > g.N)
+    return -1;
+  return caj::qtile_key_tiles(g, q0, q1, block_n, t[0], t[1], t[2], t[3]);
+}
+
+caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const void *tq,
+                            const void *tk, const void *tv, const caj_problem *prob,
+                            const caj_mask_desc *mask, void *o, void *to, float *lse, float *tlse,
+                            void *stream) {
+  if (!prob || !mask) return CAJ_ERR_INVALID_ARG;
+  const void *ins[6] = {q, k, v, tq, tk, tv};
+  for (const void *p : ins)
+    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
+  if (!o || !to || !aligned16(o) || !aligned16(to)) return CAJ_ERR_INVALID_ARG;
+  if (!lse || !tlse || !aligned4(lse) || !aligned4(tlse)) return CAJ_ERR_INVALID_ARG;
+  if (prob->B <= 0 || prob->H <= 0 || prob->N <= 0 || prob->D <= 0) return CAJ_ERR_INVALID_ARG;
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g) || g.N != prob->N) return CAJ_ERR_INVALID_ARG;
+  if (prob->dtype != CAJ_DTYPE_F32 && prob->dtype != CAJ_DTYPE_BF16) return CAJ_ERR_INVALID_ARG;
+  if (!(prob->scale >= 0.f) || std::isinf(prob->scale)) return CAJ_ERR_INVALID_ARG;
+  if (prob->D != 64 && prob->D != 128) return CAJ_ERR_UNSUPPORTED;
+  const int64_t BH = int64_t(prob->B) * prob->H;
+  if (BH > 65535 || prob->N > (1 << 20)) return CAJ_ERR_UNSUPPORTED;
+
+  caj_status st = check_device();
+  if (st != CAJ_OK) return st;
+
+  const float scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt(float(prob->D));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  if (prob->dtype == CAJ_DTYPE_F32) {
+    caj::SimtParams p{};
+    p.q = q; p.k = k; p.v = v; p.tq = tq; p.tk = tk; p.tv = tv;
+    p.o = o; p.to = to; p.lse = lse; p.tlse = tlse;
+    p.geom = g;
+    p.BH = int32_t(BH);
+    p.scale = scale;
+    cudaError_t e = caj::launch_fwd_jvp_simt_f32(p, prob->D, s);
+    return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+  }
+
+  const int32_t n_qtiles = (prob->N + caj::kBlockM - 1) / caj::kBlockM;
+  if (n_qtiles > caj::kMaxQTiles) return CAJ_ERR_UNSUPPORTED;
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+
+  // Parameters live in a heap block: the struct carries the launch order table.
+  std::unique_ptr<caj::Sm100Params> hp(new caj::Sm100Params());
+  caj::Sm100Params &p = *hp;
+  const int N = prob->N, D = prob->D;
+  bool okm = encode_map(enc, &p.tm_q, q, int(BH), N, D, caj::kBlockM) &&
+             encode_map(enc, &p.tm_tq, tq, int(BH), N, D, caj::kBlockM) &&
+             encode_map(enc, &p.tm_k, k, int(BH), N, D, caj::kBlockN) &&
+             encode_map(enc, &p.tm_tk, tk, int(BH), N, D, caj::kBlockN) &&
+             encode_map(enc, &p.tm_v, v, int(BH), N, D, caj::kBlockN) &&
+             encode_map(enc, &p.tm_tv, tv, int(BH), N, D, caj::kBlockN);
+  if (!okm) return cuda_fail(cudaErrorInvalidValue);
+  p.o = o; p.to = to; p.lse = lse; p.tlse = tlse;
+  p.geom = g;
+  p.BH = int32_t(BH);
+  p.n_qtiles = n_qtiles;
+  p.scale = scale;
+  p.scale_log2e = scale * 1.4426950408889634f;
+  p.timeout_ns = wait_timeout_ns();
+  // Launch order: query tiles by decreasing number of key tiles (ties: later first).
+  std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
+  for (int32_t t = 0; t < n_qtiles; ++t) {
+    int32_t r[4];
+    const int32_t q0 = t * caj::kBlockM, q1 = std::min(q0 + caj::kBlockM, N);
+    cost[t] = {caj::qtile_key_tiles(g, q0, q1, caj::kBlockN, r[0], r[1], r[2], r[3]), t};
+  }
+  std::sort(cost.begin(), cost.end(), [](const auto &a, const auto &b) {
+    return a.first != b.first ? a.first > b.first : a.second > b.second;
+  });
+  for (int32_t i = 0; i < n_qtiles; ++i) p.qtile_order[i] = uint16_t(cost[i].second);
+
+  cudaError_t e = caj::launch_fwd_jvp_sm100(p, D, s);
+  return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+}
+
+caj_status caj_last_device_status(void *stream) {
+  uint32_t code = 0;
+  cudaError_t e = caj::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &code);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (code != 0) {
+    g_last_device_code = code;
+    return CAJ_ERR_DEVICE_TIMEOUT;
+  }
+  return CAJ_OK;
+}
+
+uint32_t caj_last_device_error_code(void) { return g_last_device_code; }
+
+}  // extern "C"

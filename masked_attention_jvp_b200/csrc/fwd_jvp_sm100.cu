@@ -1,0 +1,541 @@
+// Fused forward + JVP of block-causal attention on B200 tensor cores (sm_100a).
+//
+// Computes, per (batch*head, 128-row query tile), the masked attention output
+// and its forward-mode tangent of the Causal-rCM paper, appendix B (eq. 42-45,
+// Algorithm 1): the online softmax of FlashAttention carries, next to the usual
+// running max m, normaliser l and output accumulator O, the JVP accumulators
+//   T = sum_j p~_j (ts_j v_j + tv_j)      (value-tangent + score-tangent terms)
+//   r = sum_j p~_j ts_j                    (row scalar)
+// all rescaled by the same online factor; after the last key tile
+//   O = O / l,  mu = r / l,  tO = T / l - mu O,  LSE = ln l + m,  tLSE = mu.
+//
+// Design (sm_100a, one CTA per query tile, 6 warps):
+//   warp 0      TMA producer: Q, tQ once; then K|tK and V|tV tiles of 64 keys
+//               through 3- and 2-deep shared-memory rings (128-byte swizzle).
+//   warp 1      tcgen05 MMA issuer (one thread), also owns the TMEM allocation:
+//                 [S | tS_1] = Q [K ; tK]^T        (one N=128 MMA per k-step)
+//                 tS += tQ K^T                      (N=64)
+//                 [O | T] += P [V | tV]             (A = P from TMEM, N=2D)
+//                 T += (P o tS) V                   (A = P o tS from TMEM, N=D)
+//               S/tS are double-buffered in TMEM so the scores of tile j+1 are
+//               computed while tile j's softmax runs.
+//   warps 2-5   softmax / epilogue, one thread per query row: TMEM -> registers,
+//               mask (only where a tile is not entirely visible to the row),
+//               exp2-domain online softmax with a lazily updated max, bf16 P and
+//               P o tS written back over the scores in TMEM, and the final
+//               normalisation and JVP epilogue.
+// TMEM (512 columns x 128 lanes, fp32): O [0,D) | T [D,2D) | S/tS buffer 0 |
+// S/tS buffer 1, each buffer S [64 cols] then tS [64 cols].
+//
+// Every wait on an mbarrier is bounded by a time limit; on expiry the kernel
+// records an error code in a device word, drains its own in-flight copies and
+// MMAs, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "mask_schedule.h"
+#include "ptx_sm100.cuh"
+
+namespace caj {
+
+__device__ uint32_t g_device_error = 0;
+
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = kBlockM;  // query rows per tile
+constexpr int BN = kBlockN;  // keys per tile
+constexpr int kThreads = 192;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale once the max grew by 2^8
+
+template <int D>
+struct Cfg {
+  static constexpr int NB = D / 64;                    // 128-byte column blocks per row
+  static constexpr int QBLK = BM * 128;                // one column block of a Q tile
+  static constexpr int Q_BYTES = NB * QBLK;
+  static constexpr int KBLK = 2 * BN * 128;            // one column block of [K ; tK]
+  static constexpr int KT_STAGE = NB * KBLK;
+  static constexpr int VBLK = BN * 128;                // one column block of V (or tV)
+  static constexpr int V_STAGE = 2 * NB * VBLK;        // V blocks, then tV blocks
+  static constexpr int KS = (D == 128) ? 3 : 4;
+  static constexpr int VS = (D == 128) ? 2 : 4;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_TQ = Q_BYTES;
+  static constexpr int OFF_KT = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_KT + KS * KT_STAGE;
+  static constexpr int OFF_BAR = OFF_V + VS * V_STAGE;
+  // barriers: q_full, kv_full[KS], kv_empty[KS], v_full[VS], v_empty[VS],
+  //           s_full[2], p_full[2], o_done[2], drain
+  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  // tensor memory columns
+  static constexpr uint32_t COL_O = 0;
+  static constexpr uint32_t COL_T = D;
+  static constexpr uint32_t COL_S0 = 2 * D;
+  static constexpr uint32_t BUF_COLS = 2 * BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(COL_S0 + 2 * BUF_COLS <= TMEM_COLS, "tensor memory overflow");
+  static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+  static constexpr uint32_t Q_TX = 2 * Q_BYTES;
+  static constexpr uint32_t KT_TX = KT_STAGE;
+  static constexpr uint32_t V_TX = V_STAGE;
+};
+
+struct Barriers {
+  uint32_t q_full, kv_full, kv_empty, v_full, v_empty, s_full, p_full, o_done, drain;
+};
+
+template <int D>
+__device__ __forceinline__ Barriers make_barriers(uint32_t base) {
+  using C = Cfg<D>;
+  Barriers b;
+  b.q_full = base;
+  b.kv_full = base + 8;
+  b.kv_empty = b.kv_full + 8 * C::KS;
+  b.v_full = b.kv_empty + 8 * C::KS;
+  b.v_empty = b.v_full + 8 * C::VS;
+  b.s_full = b.v_empty + 8 * C::VS;
+  b.p_full = b.s_full + 16;
+  b.o_done = b.p_full + 16;
+  b.drain = b.o_done + 16;
+  return b;
+}
+
+// Record the first device error and raise the CTA's abort flag.
+__device__ __noinline__ void raise_error(volatile int *abort_flag, uint32_t code) {
+  atomicCAS(&g_device_error, 0u, code);
+  *abort_flag = 1;
+}
+
+// Wait for completion of the phase with parity `parity`. Gives up (returns
+// false) when the CTA has aborted or after `timeout_ns`, recording `site`.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile int *abort_flag, uint64_t timeout_ns,
+                                             uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1; it < 0x40000000u; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        raise_error(abort_flag, kErrTimeoutBase | site);
+        return false;
+      }
+    }
+  }
+  raise_error(abort_flag, kErrTimeoutBase | site);
+  return false;
+}
+
+// Same, ignoring the abort flag: used only to drain this CTA's own in-flight
+// copies and MMAs before it releases shared and tensor memory.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1; it < 0x40000000u; ++it) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((it & 31u) == 0 && globaltimer_ns() - t0 > timeout_ns) return;
+  }
+}
+
+// Key tile index of the j-th visited tile.
+__device__ __forceinline__ int32_t tile_at(int32_t j, int32_t t0, int32_t n0, int32_t t2) {
+  return j < n0 ? t0 + j : t2 + (j - n0);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t *sgen = smem_raw + (sbase - raw);
+  const Barriers bar = make_barriers<D>(sbase + C::OFF_BAR);
+  volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sgen + C::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Work item: heaviest query tiles first, heads fastest.
+  const int32_t qt = p.qtile_order[blockIdx.x / p.BH];
+  const int32_t bh = blockIdx.x % p.BH;
+  const int32_t q0 = qt * BM;
+  const int32_t q1 = min(q0 + BM, p.geom.N);
+  int32_t t0, t1, t2, t3;
+  const int32_t ntiles = qtile_key_tiles(p.geom, q0, q1, BN, t0, t1, t2, t3);
+  const int32_t n0 = t1 - t0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar.q_full, 1);
+    for (int s = 0; s < C::KS; ++s) {
+      mbar_init(bar.kv_full + 8 * s, 1);
+      mbar_init(bar.kv_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < C::VS; ++s) {
+      mbar_init(bar.v_full + 8 * s, 1);
+      mbar_init(bar.v_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar.s_full + 8 * b, 1);
+      mbar_init(bar.p_full + 8 * b, 4);  // one arrival per softmax warp
+      mbar_init(bar.o_done + 8 * b, 1);
+    }
+    mbar_init(bar.drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&p.tm_q);
+      prefetch_tmap(&p.tm_k);
+      prefetch_tmap(&p.tm_v);
+      const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
+      mbar_arrive_expect_tx(bar.q_full, C::Q_TX);
+      for (int c = 0; c < C::NB; ++c) {
+        tma_load_3d(sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
+        tma_load_3d(stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
+      }
+      int32_t k_issued = 0, v_issued = 0;
+      bool ok = true;
+      auto issue_k = [&](int32_t j) -> bool {
+        const int s = j % C::KS;
+        if (j >= C::KS &&
+            !wait_bounded(bar.kv_empty + 8 * s, ((j / C::KS) - 1) & 1, abort_flag, p.timeout_ns, 1))
+          return false;
+        const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
+        const uint32_t dst = sbase + C::OFF_KT + s * C::KT_STAGE;
+        const uint32_t fb = bar.kv_full + 8 * s;
+        mbar_arrive_expect_tx(fb, C::KT_TX);
+        for (int c = 0; c < C::NB; ++c) {
+          tma_load_3d(dst + c * C::KBLK, &p.tm_k, fb, c * 64, key0, bh);
+          tma_load_3d(dst + c * C::KBLK + BN * 128, &p.tm_tk, fb, c * 64, key0, bh);
+        }
+        k_issued = j + 1;
+        return true;
+      };
+      auto issue_v = [&](int32_t j) -> bool {
+        const int s = j % C::VS;
+        if (j >= C::VS &&
+            !wait_bounded(bar.v_empty + 8 * s, ((j / C::VS) - 1) & 1, abort_flag, p.timeout_ns, 2))
+          return false;
+        const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
+        const uint32_t dst = sbase + C::OFF_V + s * C::V_STAGE;
+        const uint32_t fb = bar.v_full + 8 * s;
+        mbar_arrive_expect_tx(fb, C::V_TX);
+        for (int c = 0; c < C::NB; ++c) {
+          tma_load_3d(dst + c * C::VBLK, &p.tm_v, fb, c * 64, key0, bh);
+          tma_load_3d(dst + (C::NB + c) * C::VBLK, &p.tm_tv, fb, c * 64, key0, bh);
+        }
+        v_issued = j + 1;
+        return true;
+      };
+      // K runs one tile ahead of V: the scores of tile j+1 are needed before
+      // the value products of tile j.
+      ok = issue_k(0);
+      for (int32_t j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles) ok = issue_k(j + 1);
+        if (ok) ok = issue_v(j);
+      }
+      // Drain: every copy this thread issued must land before the CTA exits.
+      drain_wait(bar.q_full, 0, p.timeout_ns);
+      for (int32_t j = (k_issued > C::KS ? k_issued - C::KS : 0); j < k_issued; ++j)
+        drain_wait(bar.kv_full + 8 * (j % C::KS), (j / C::KS) & 1, p.timeout_ns);
+      for (int32_t j = (v_issued > C::VS ? v_issued - C::VS : 0); j < v_issued; ++j)
+        drain_wait(bar.v_full + 8 * (j % C::VS), (j / C::VS) & 1, p.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_S = idesc_bf16_f32(BM, 2 * BN, 0);   // Q [K;tK]^T
+      constexpr uint32_t ID_TS = idesc_bf16_f32(BM, BN, 0);      // tQ K^T
+      constexpr uint32_t ID_OT = idesc_bf16_f32(BM, 2 * D, 1);   // P [V|tV]
+      constexpr uint32_t ID_T = idesc_bf16_f32(BM, D, 1);        // (P o tS) V
+      const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
+      bool ok = wait_bounded(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
+      auto issue_scores = [&](int32_t j) -> bool {
+        const int s = j % C::KS;
+        if (!wait_bounded(bar.kv_full + 8 * s, (j / C::KS) & 1, abort_flag, p.timeout_ns, 4))
+          return false;
+        tc_fence_after();
+        const uint32_t kt = sbase + C::OFF_KT + s * C::KT_STAGE;
+        const uint32_t dS = tmem + C::COL_S0 + (j & 1) * C::BUF_COLS;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
+          const uint64_t a_q = sdesc_sw128(sq + (kk >> 2) * C::QBLK + koff, 16, 1024);
+          const uint64_t a_tq = sdesc_sw128(stq + (kk >> 2) * C::QBLK + koff, 16, 1024);
+          const uint64_t b_k = sdesc_sw128(kt + (kk >> 2) * C::KBLK + koff, 16, 1024);
+          mma_ss(dS, a_q, b_k, ID_S, kk > 0 ? 1u : 0u);
+          mma_ss(dS + BN, a_tq, b_k, ID_TS, 1u);
+        }
+        tc_commit(bar.kv_empty + 8 * s);
+        tc_commit(bar.s_full + 8 * (j & 1));
+        return true;
+      };
+      auto issue_values = [&](int32_t i) -> bool {
+        const int s = i % C::VS;
+        if (!wait_bounded(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5))
+          return false;
+        if (!wait_bounded(bar.v_full + 8 * s, (i / C::VS) & 1, abort_flag, p.timeout_ns, 6))
+          return false;
+        tc_fence_after();
+        const uint32_t vt = sbase + C::OFF_V + s * C::V_STAGE;
+        const uint32_t aP = tmem + C::COL_S0 + (i & 1) * C::BUF_COLS;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // MN-major B: 64-element column blocks C::VBLK apart, 8-key groups 1 KiB apart.
+          const uint64_t b_v = sdesc_sw128(vt + kk * 16 * 128, C::VBLK, 1024);
+          mma_ts(tmem + C::COL_O, aP + kk * 8, b_v, ID_OT, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::COL_T, aP + BN + kk * 8, b_v, ID_T, 1u);
+        }
+        tc_commit(bar.v_empty + 8 * s);
+        tc_commit(bar.o_done + 8 * (i & 1));
+        return true;
+      };
+      for (int32_t j = 0; ok && j <= ntiles; ++j) {
+        if (j < ntiles) ok = issue_scores(j);
+        if (ok && j >= 1) ok = issue_values(j - 1);
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      tc_commit(bar.drain);
+      drain_wait(bar.drain, 0, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------- softmax + epilogue
+    const int sub = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = sub * 32 + lane;          // query row within the tile
+    const int32_t q = q0 + row;
+    const uint32_t lane_addr = tmem + (uint32_t(sub * 32) << 16);
+    int32_t a0, b0, a1, b1;
+    if (q < p.geom.N) {
+      row_key_ranges(p.geom, q, a0, b0, a1, b1);
+    } else {  // padding row past the sequence end: keep it finite, never stored
+      a0 = 0;
+      b0 = p.geom.N;
+      a1 = b1 = 0;
+    }
+    const float sl2 = p.scale_log2e;
+    const float scale = p.scale;
+    float m_run = -INFINITY;  // running max of s * scale * log2(e), possibly stale by < 2^8
+    float l_run = 0.f, r_run = 0.f;
+    bool ok = true;
+
+    for (int32_t j = 0; j < ntiles; ++j) {
+      const int b = j & 1;
+      const bool got = wait_bounded(bar.s_full + 8 * b, (j >> 1) & 1, abort_flag, p.timeout_ns, 7);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int32_t k0 = tile_at(j, t0, n0, t2) * BN;
+      const uint32_t cS = lane_addr + C::COL_S0 + b * C::BUF_COLS;
+      float s[BN];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(cS, r0);
+        tmem_ld32(cS + 32, r1);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(r0[i]);
+          s[32 + i] = __uint_as_float(r1[i]);
+        }
+      }
+      // Mask only where this tile is not entirely inside the row's key ranges.
+      const bool full = (k0 >= a0 && k0 + BN <= b0) || (k0 >= a1 && k0 + BN <= b1);
+      uint32_t vis_lo = 0xffffffffu, vis_hi = 0xffffffffu;
+      if (!full) {
+        vis_lo = vis_hi = 0;
+#pragma unroll
+        for (int i = 0; i < BN; ++i) {
+          const int32_t key = k0 + i;
+          const bool v = (key >= a0 && key < b0) || (key >= a1 && key < b1);
+          if (i < 32) vis_lo |= uint32_t(v) << i;
+          else vis_hi |= uint32_t(v) << (i - 32);
+          s[i] = v ? s[i] : -INFINITY;
+        }
+      }
+      float tmax = s[0];
+#pragma unroll
+      for (int i = 1; i < BN; ++i) tmax = fmaxf(tmax, s[i]);
+      const float m_tile = tmax * sl2;  // -inf if the row sees nothing here
+      // Lazy rescale: keep the old max unless the new one exceeds it by 2^8.
+      const bool grow = m_tile > m_run + kRescaleThreshold;
+      const bool had_acc = m_run != -INFINITY;  // accumulators hold non-zero data
+      float alpha = 1.f;
+      if (grow) {
+        alpha = had_acc ? ex2(m_run - m_tile) : 0.f;
+        l_run *= alpha;
+        r_run *= alpha;
+        m_run = m_tile;
+      }
+      if (__any_sync(0xffffffffu, grow && had_acc) && j > 0) {
+        // O and T of this warp's rows must be scaled by alpha; wait until the
+        // value MMAs of the previous tile have landed.
+        const int pb = (j - 1) & 1;
+        const bool g2 =
+            wait_bounded(bar.o_done + 8 * pb, ((j - 1) >> 1) & 1, abort_flag, p.timeout_ns, 8);
+        if (!__all_sync(0xffffffffu, g2)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 2 * D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + C::COL_O + c, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(lane_addr + C::COL_O + c, r);
+        }
+        tmem_wait_st();
+      }
+      const float ref = (m_run == -INFINITY) ? 0.f : m_run;
+      // P = 2^(s*scale*log2e - ref), rounded to bf16 and written over S.
+      float lsum = 0.f;
+#pragma unroll
+      for (int i = 0; i < BN; ++i) {
+        s[i] = ex2(fmaf(s[i], sl2, -ref));
+        lsum += s[i];
+      }
+      l_run += lsum;
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(s[2 * i], s[2 * i + 1]);
+        tmem_st32(cS, pk);
+      }
+      // P o tS (scaled), rounded to bf16 and written over tS; r += sum p ts.
+      float rsum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t tr[32];
+        tmem_ld32(cS + BN + 32 * h, tr);
+        const uint32_t vis = h ? vis_hi : vis_lo;
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float ta = __uint_as_float(tr[2 * i]) * scale;
+          float tb = __uint_as_float(tr[2 * i + 1]) * scale;
+          ta = ((vis >> (2 * i)) & 1u) ? ta : 0.f;
+          tb = ((vis >> (2 * i + 1)) & 1u) ? tb : 0.f;
+          const float pa = s[32 * h + 2 * i] * ta, pb = s[32 * h + 2 * i + 1] * tb;
+          rsum += pa + pb;
+          pk[i] = pack_bf16(pa, pb);
+        }
+        tmem_st16(cS + BN + 16 * h, pk);
+      }
+      r_run += rsum;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.p_full + 8 * b);
+    }
+
+    if (ok && ntiles > 0) {
+      const int32_t last = ntiles - 1;
+      const bool got =
+          wait_bounded(bar.o_done + 8 * (last & 1), (last >> 1) & 1, abort_flag, p.timeout_ns, 9);
+      if (__all_sync(0xffffffffu, got)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_run;
+        const float mu = r_run * inv_l;
+        const bool store = q < p.geom.N;
+        const size_t rowoff = (size_t(bh) * p.geom.N + (store ? q : 0)) * D;
+        uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
+        uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t ro[32], rt[32];
+          tmem_ld32(lane_addr + C::COL_O + c, ro);
+          tmem_ld32(lane_addr + C::COL_T + c, rt);
+          uint32_t po[16], pt[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float oa = __uint_as_float(ro[2 * i]) * inv_l;
+            const float ob = __uint_as_float(ro[2 * i + 1]) * inv_l;
+            const float ta = fmaf(__uint_as_float(rt[2 * i]), inv_l, -mu * oa);
+            const float tb = fmaf(__uint_as_float(rt[2 * i + 1]), inv_l, -mu * ob);
+            po[i] = pack_bf16(oa, ob);
+            pt[i] = pack_bf16(ta, tb);
+          }
+          if (store) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              orow[c / 8 + v] = make_uint4(po[4 * v], po[4 * v + 1], po[4 * v + 2], po[4 * v + 3]);
+              torow[c / 8 + v] = make_uint4(pt[4 * v], pt[4 * v + 1], pt[4 * v + 2], pt[4 * v + 3]);
+            }
+          }
+        }
+        if (store) {
+          const size_t ri = size_t(bh) * p.geom.N + q;
+          p.lse[ri] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+          p.tlse[ri] = mu;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_impl(const Sm100Params &p, cudaStream_t stream) {
+  using C = Cfg<D>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
+  fwd_jvp_sm100_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream) {
+  if (D == 128) return launch_impl<128>(p, stream);
+  if (D == 64) return launch_impl<64>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t read_and_clear_device_error(cudaStream_t stream, uint32_t *out) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  uint32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return e;
+  }
+  *out = v;
+  return cudaSuccess;
+}
+
+}  // namespace caj

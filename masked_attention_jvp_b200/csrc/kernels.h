@@ -1,0 +1,54 @@
+// Internal launch interface between the C-ABI front end (api.cpp) and the CUDA
+// translation units. Not part of the public header.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mask_schedule.h"
+
+namespace caj {
+
+// Query-tile height of both kernels' work decomposition (rows per tile).
+constexpr int kBlockM = 128;
+// Key-tile width of the tensor-core kernel.
+constexpr int kBlockN = 64;
+// Largest number of query tiles per head the launch order table can hold.
+constexpr int kMaxQTiles = 4096;
+
+// Device error word values (first error wins). Low byte: where a wait gave up.
+enum DeviceError : uint32_t {
+  kErrNone = 0,
+  kErrTimeoutBase = 0x100,  // | wait site
+};
+
+struct Sm100Params {
+  CUtensorMap tm_q, tm_tq, tm_k, tm_tk, tm_v, tm_tv;  // 3-D maps over [B*H, N, D]
+  void *o, *to;          // [B*H, N, D] bf16
+  float *lse, *tlse;     // [B*H, N]
+  MaskGeom geom;
+  int32_t BH;
+  int32_t n_qtiles;
+  float scale;           // softmax scale
+  float scale_log2e;     // scale * log2(e)
+  uint64_t timeout_ns;   // bounded-wait limit
+  uint16_t qtile_order[kMaxQTiles];  // heaviest query tiles first
+};
+
+struct SimtParams {
+  const void *q, *k, *v, *tq, *tk, *tv;
+  void *o, *to;
+  float *lse, *tlse;
+  MaskGeom geom;
+  int32_t BH;
+  float scale;
+};
+
+// Each returns the launch's cudaError_t (cudaSuccess when enqueued).
+cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream);
+cudaError_t launch_fwd_jvp_simt_f32(const SimtParams &p, int D, cudaStream_t stream);
+
+// Device error word access (defined next to the kernels that write it).
+cudaError_t read_and_clear_device_error(cudaStream_t stream, uint32_t *out);
+
+}  // namespace caj

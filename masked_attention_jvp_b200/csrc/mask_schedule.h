@@ -1,0 +1,95 @@
+// Closed-form block-causal mask geometry and tile schedule, usable on host and
+// device.
+//
+// The mask is the teacher-forcing / block-causal family of the Causal-rCM paper
+// (section 3.1.1, eq. 8; Table 2 legend; section 4 chunk modes). Appendix B
+// represents such masks as a short list of query groups, each with a few
+// allowed key ranges, and streams only those ranges; the same schedule serves
+// the primal and the tangent. Here that list is not stored: every row's key
+// ranges and every query tile's key-tile ranges follow from four integers.
+#pragma once
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define CAJ_HD __host__ __device__ __forceinline__
+#else
+#define CAJ_HD inline
+#endif
+
+namespace caj {
+
+struct MaskGeom {
+  int32_t G;   // tokens per chunk (frames_per_chunk * tokens_per_frame)
+  int32_t L;   // tokens of one copy of the video (n_frames * tokens_per_frame)
+  int32_t N;   // sequence length (L, or 2L for the teacher-forcing layout)
+  int32_t tf;  // 1 = [clean | noisy] teacher-forcing layout
+};
+
+// Keys visible to query `q`: [a0, b0) U [a1, b1), both possibly empty.
+//   plain / clean query in chunk j: [0, (j+1) G)
+//   noisy query in chunk j:         [0, j G) U [L + j G, L + (j+1) G)
+CAJ_HD void row_key_ranges(const MaskGeom &m, int32_t q, int32_t &a0, int32_t &b0,
+                           int32_t &a1, int32_t &b1) {
+  if (!m.tf || q < m.L) {
+    a0 = 0;
+    b0 = (q / m.G + 1) * m.G;
+    a1 = b1 = 0;
+  } else {
+    int32_t j = (q - m.L) / m.G;
+    a0 = 0;
+    b0 = j * m.G;
+    a1 = m.L + j * m.G;
+    b1 = a1 + m.G;
+  }
+}
+
+// Key tiles of width bn that query rows [q0, q1) touch, as up to two ascending
+// disjoint tile ranges [t0, t1) U [t2, t3). Returns the number of tiles.
+CAJ_HD int32_t qtile_key_tiles(const MaskGeom &m, int32_t q0, int32_t q1, int32_t bn,
+                               int32_t &t0, int32_t &t1, int32_t &t2, int32_t &t3) {
+  // Union of the rows' ranges: one prefix [0, pre) plus, for noisy rows, one
+  // band [lo, hi) inside the noisy copy.
+  int32_t pre = 0, lo = 0, hi = 0;
+  const int32_t clean_end = m.tf ? m.L : m.N;
+  if (q0 < clean_end) {
+    int32_t last = (q1 < clean_end ? q1 : clean_end) - 1;
+    pre = (last / m.G + 1) * m.G;
+  }
+  if (m.tf && q1 > m.L) {
+    int32_t first = q0 > m.L ? q0 : m.L;
+    int32_t j0 = (first - m.L) / m.G, j1 = (q1 - 1 - m.L) / m.G;
+    int32_t noisy_pre = j1 * m.G;  // the last noisy row's clean history is the widest
+    if (noisy_pre > pre) pre = noisy_pre;
+    lo = m.L + j0 * m.G;
+    hi = m.L + (j1 + 1) * m.G;
+  }
+  t0 = 0;
+  t1 = (pre + bn - 1) / bn;
+  if (hi > lo) {
+    t2 = lo / bn;
+    t3 = (hi + bn - 1) / bn;
+    if (t2 <= t1) {  // the prefix and the band share or touch a tile: merge
+      if (t3 > t1) t1 = t3;
+      t2 = t3 = t1;
+    }
+  } else {
+    t2 = t3 = t1;
+  }
+  if (t1 == 0) {  // no prefix (noisy rows of chunk 0 only): the band alone
+    t0 = t2;
+    t1 = t3;
+    t2 = t3 = t1;
+  }
+  return (t1 - t0) + (t3 - t2);
+}
+
+// Visible (query, key) pairs of one head: n chunks of G tokens; chunk j of the
+// plain layout sees j+1 chunks (G^2 n(n+1)/2 in all); the teacher-forcing
+// layout adds the same count again for the noisy copy.
+CAJ_HD int64_t visible_pairs(const MaskGeom &m) {
+  int64_t n = m.L / m.G, G = m.G;
+  int64_t half = G * G * n * (n + 1) / 2;
+  return m.tf ? 2 * half : half;
+}
+
+}  // namespace caj

@@ -1,0 +1,152 @@
+"""Host-side checks of libcausaljvp that need no GPU: the library loads and
+exports every symbol its header declares, the closed-form mask / tile schedule
+matches brute force over the oracle's independent visibility rule, and argument
+validation rejects bad calls before anything is launched."""
+import ctypes
+import os
+import random
+import re
+
+import pytest
+import torch
+
+import oracle
+import masked_attention_jvp_b200 as caj
+from masked_attention_jvp_b200 import _lib
+from masked_attention_jvp_b200.workloads import MaskDesc, WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MASKS = [MaskDesc(3, 1, 4, 0), MaskDesc(2, 2, 4, 0), MaskDesc(3, 1, 3, 1), MaskDesc(2, 3, 6, 1),
+         MaskDesc(1, 1, 7, 0), MaskDesc(5, 1, 1, 0), MaskDesc(37, 1, 5, 1), MaskDesc(100, 1, 3, 0),
+         MaskDesc(13, 3, 6, 1), MaskDesc(64, 1, 4, 1), MaskDesc(1, 1, 130, 1)]
+
+
+def test_header_symbols_are_exported():
+    hdr = open(os.path.join(ROOT, "include", "causaljvp.h")).read()
+    declared = sorted(set(re.findall(r"\b(caj_[a-z_]+)\s*\(", hdr)))
+    assert declared == sorted(_lib.EXPORTED)
+    L = _lib.lib()
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings():
+    assert _lib.lib().caj_version() >= 100
+    names = [_lib.status_string(i) for i in range(5)]
+    assert names == ["CAJ_OK", "CAJ_ERR_INVALID_ARG", "CAJ_ERR_UNSUPPORTED", "CAJ_ERR_CUDA",
+                     "CAJ_ERR_DEVICE_TIMEOUT"]
+    assert _lib.status_string(99) == "CAJ_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("mask", MASKS)
+def test_visible_pairs_matches_brute_force(mask):
+    assert caj.visible_pairs(mask) == oracle.visible_pairs(mask)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_visible_pairs_of_the_workloads(name):
+    w = WORKLOADS[name]
+    m = w.mask
+    G, n = m.frames_per_chunk * m.tokens_per_frame, m.n_frames // m.frames_per_chunk
+    half = G * G * n * (n + 1) // 2
+    assert caj.visible_pairs(m) == (2 * half if m.tf_layout else half)
+
+
+@pytest.mark.parametrize("mask", MASKS)
+def test_row_ranges_match_oracle_visibility(mask):
+    N = mask.seq_len
+    for i in range(N):
+        (a0, b0), (a1, b1) = caj.row_key_ranges(mask, i)
+        got = set(range(a0, b0)) | set(range(a1, b1))
+        want = {j for j in range(N) if oracle.visible(mask, i, j)}
+        assert got == want, (mask, i)
+
+
+@pytest.mark.parametrize("mask", MASKS)
+@pytest.mark.parametrize("bm,bn", [(128, 64), (16, 8), (7, 5), (32, 64)])
+def test_query_tile_schedule_matches_brute_force(mask, bm, bn):
+    """The kernel visits exactly the key tiles some row of the query tile can see."""
+    N = mask.seq_len
+    for q0 in range(0, N, bm):
+        q1 = min(q0 + bm, N)
+        n, (t0, t1), (t2, t3) = caj.qtile_key_tiles(mask, q0, q1, bn)
+        assert t0 <= t1 <= t2 <= t3
+        tiles = list(range(t0, t1)) + list(range(t2, t3))
+        assert n == len(tiles)
+        want = sorted({j // bn for i in range(q0, q1) for j in range(N) if oracle.visible(mask, i, j)})
+        assert tiles == want, (mask, q0, q1, bn)
+
+
+@pytest.mark.parametrize("name", [n for n in WORKLOADS if n != "tiny_framewise_fp32"])
+def test_schedule_at_full_size_covers_every_row(name):
+    """At the workloads' sizes: every row's key ranges lie inside its tile's
+    visited tiles, and the visited tiles hold no tile that no row needs (sampled)."""
+    m = WORKLOADS[name].mask
+    N = m.seq_len
+    rng = random.Random(5)
+    tiles_q = list(range((N + 127) // 128))
+    for qt in rng.sample(tiles_q, 40) + [0, len(tiles_q) - 1]:
+        q0, q1 = qt * 128, min(qt * 128 + 128, N)
+        n, (t0, t1), (t2, t3) = caj.qtile_key_tiles(m, q0, q1, 64)
+        tiles = set(range(t0, t1)) | set(range(t2, t3))
+        needed = set()
+        for i in range(q0, q1):
+            (a0, b0), (a1, b1) = caj.row_key_ranges(m, i)
+            for a, b in ((a0, b0), (a1, b1)):
+                if b > a:
+                    needed |= set(range(a // 64, (b + 63) // 64))
+        assert tiles == needed
+
+
+def _call(q=0x10000, o=0x20000, lse=0x30000, prob=None, mask=None):
+    prob = prob or _lib.ProblemC(1, 2, 64, 64, _lib.CAJ_DTYPE_BF16, 0.0)
+    mask = mask or _lib.MaskDescC(16, 1, 4, 0)
+    vp = ctypes.c_void_p
+    return _lib.lib().caj_attn_fwd_jvp(vp(q), vp(q), vp(q), vp(q), vp(q), vp(q),
+                                       ctypes.byref(prob), ctypes.byref(mask),
+                                       vp(o), vp(o), vp(lse), vp(lse), vp(0))
+
+
+def test_argument_validation_launches_nothing():
+    P, M = _lib.ProblemC, _lib.MaskDescC
+    bf = _lib.CAJ_DTYPE_BF16
+    INV, UNS = _lib.CAJ_ERR_INVALID_ARG, _lib.CAJ_ERR_UNSUPPORTED
+    assert _call(q=0) == INV                                   # null input
+    assert _call(q=0x10008) == INV                             # misaligned input
+    assert _call(o=0x20004) == INV                             # misaligned output
+    assert _call(lse=0x30002) == INV                           # misaligned lse
+    assert _call(prob=P(1, 2, 65, 64, bf, 0.0)) == INV         # N != mask length
+    assert _call(prob=P(0, 2, 64, 64, bf, 0.0)) == INV         # empty batch
+    assert _call(prob=P(1, 2, 64, 64, 7, 0.0)) == INV          # unknown dtype
+    assert _call(prob=P(1, 2, 64, 64, bf, -1.0)) == INV        # negative scale
+    assert _call(prob=P(1, 2, 64, 64, bf, float("nan"))) == INV
+    assert _call(mask=M(16, 3, 4, 0)) == INV                   # frames % chunk != 0
+    assert _call(mask=M(16, 1, 4, 2)) == INV                   # bad layout flag
+    assert _call(mask=M(0, 1, 4, 0)) == INV                    # empty frame
+    assert _call(prob=P(1, 2, 128, 64, bf, 0.0), mask=M(16, 1, 4, 1)) != INV  # TF: N = 2L
+    assert _call(prob=P(1, 2, 64, 96, bf, 0.0)) == UNS         # head dim not built
+    assert _call(prob=P(700, 100, 64, 64, bf, 0.0)) == UNS     # too many heads
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_valid_call_without_gpu_reports_cuda_error():
+    assert _call() == _lib.CAJ_ERR_CUDA
+    assert len(_lib.lib().caj_last_cuda_error()) > 0
+
+
+def test_mask_queries_reject_bad_arguments():
+    M = _lib.MaskDescC
+    L = _lib.lib()
+    assert L.caj_validate_mask(ctypes.byref(M(16, 1, 4, 0)), 64) == _lib.CAJ_OK
+    assert L.caj_validate_mask(ctypes.byref(M(16, 1, 4, 1)), 64) == _lib.CAJ_ERR_INVALID_ARG
+    assert L.caj_visible_pairs(ctypes.byref(M(16, 2, 3, 0))) == -1
+    r = (ctypes.c_int32 * 4)()
+    assert L.caj_row_key_ranges(ctypes.byref(M(4, 1, 2, 0)), 8, r) == _lib.CAJ_ERR_INVALID_ARG
+    assert L.caj_qtile_key_tiles(ctypes.byref(M(4, 1, 2, 0)), 4, 4, 64, r) == -1
+    assert L.caj_qtile_key_tiles(ctypes.byref(M(4, 1, 2, 0)), 0, 9, 64, r) == -1
+
+
+def test_flops_count():
+    m = WORKLOADS["wan1.3b_tf_framewise"].mask
+    assert caj.flops(1, 12, 128, m) == 12 * 128 * 1_124_323_200 * 12
