@@ -154,6 +154,34 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm
+def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
+    """Same metric through the public API from pinned host buffers: every step
+    copies the six inputs host->device and the four outputs device->host."""
+    import masked_attention_jvp_b200 as caj
+    pinned = [t.pin_memory() for t in host]
+    h2d = sum(t.numel() * t.element_size() for t in pinned)
+    n_rows = w.B * w.H * w.N
+    d2h = 2 * n_rows * w.D * pinned[0].element_size() + 2 * n_rows * 4
+    steps = max(1, min(args.steps, 5))
+    caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)  # warm the host path once
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * fl * steps / (ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
 def bench_gpu(args, rank, world, local_rank):
     import masked_attention_jvp_b200 as caj
 
@@ -202,26 +230,9 @@ def bench_gpu(args, rank, world, local_rank):
     value = world * fl * args.steps / (total_ms / 1e3) / 1e12
 
     # end to end through the public API with pinned host buffers
-    pinned = [t.pin_memory() for t in host]
-    h2d = sum(t.numel() * t.element_size() for t in pinned)
-    d2h = 2 * o.numel() * o.element_size() + 2 * lse.numel() * 4
-    e2e_steps = max(1, min(args.steps, 5))
-    caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)  # warm the host path once
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * fl * e2e_steps / (e2e_ms / 1e3) / 1e12
-
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_e2e(args, w, host, fl, world, stream, dev, barrier)
     if rank != 0:
         return None
     peaks, src = load_peaks()
@@ -238,8 +249,7 @@ def bench_gpu(args, rank, world, local_rank):
         "pct_of_dense_bf16_peak": round(100.0 * value / world / DENSE_BF16_SPEC_TFLOPS, 2),
         "ms_per_step_min": round(min(per), 4), "ms_per_step_median": round(statistics.median(per), 4),
         "clocks": clocks,
-        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "e2e": e2e,
         "gpu_launches": args.steps,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
@@ -293,6 +303,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

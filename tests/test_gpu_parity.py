@@ -28,7 +28,10 @@ def rel_fro(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
 
 
-def check_rows(got, ref, dtype, what=""):
+def check_rows(got, ref, dtype, what="", maxabs_relative=False):
+    """maxabs_relative: for inputs outside the workloads' distributions (larger
+    scale or larger scores, hence larger outputs) the bf16 max-abs bound is taken
+    relative to the largest reference magnitude."""
     o, to, lse, tlse = [np.asarray(x, np.float64) for x in got]
     ro, rto, rlse, rtlse = ref
     t = TOL[dtype]
@@ -41,8 +44,10 @@ def check_rows(got, ref, dtype, what=""):
     assert errs["tlse_fro"] <= t["fro"], (what, errs)
     assert errs["lse_max"] <= t["lse"], (what, errs)
     if t["maxabs"] is not None:
-        assert errs["o_max"] <= t["maxabs"], (what, errs)
-        assert errs["to_max"] <= t["maxabs"], (what, errs)
+        o_lim = t["maxabs"] * (max(1.0, float(np.max(np.abs(ro)))) if maxabs_relative else 1.0)
+        to_lim = t["maxabs"] * (max(1.0, float(np.max(np.abs(rto)))) if maxabs_relative else 1.0)
+        assert errs["o_max"] <= o_lim, (what, errs)
+        assert errs["to_max"] <= to_lim, (what, errs, to_lim)
     return errs
 
 
@@ -61,11 +66,11 @@ def gather(outs, rows, D):
             lse.reshape(-1)[idx].cpu().numpy(), tlse.reshape(-1)[idx].cpu().numpy())
 
 
-def full_check(w: Workload):
+def full_check(w: Workload, maxabs_relative=False):
     ins, outs = run_gpu(w)
     ref = oracle.attn_fwd_jvp_rows(*[t.cpu() for t in ins], w.mask, scale=w.scale)
     rows = torch.arange(w.B * w.H * w.N)
-    return check_rows(gather(outs, rows, w.D), ref, w.dtype, w.name)
+    return check_rows(gather(outs, rows, w.D), ref, w.dtype, w.name, maxabs_relative)
 
 
 # --------------------------------------------------------------- small, full outputs
@@ -102,13 +107,13 @@ def test_small_shapes_full(case, D, dtype):
 @pytest.mark.parametrize("scale", [0.05, 0.3])
 def test_explicit_scale(scale):
     w = Workload("scaled", 1, 2, 128, MaskDesc(50, 1, 6, 1), torch.bfloat16, seed=7, scale=scale)
-    full_check(w)
+    full_check(w, maxabs_relative=True)
 
 
 def test_large_values_exercise_rescaling():
     """std 3 scores make the running max move by more than 2^8 between tiles."""
     w = Workload("wide", 1, 2, 128, MaskDesc(300, 1, 4, 1), torch.bfloat16, seed=8, std_qkv=3.0)
-    full_check(w)
+    full_check(w, maxabs_relative=True)
 
 
 # ------------------------------------------------------ full-size workloads, sampled
