@@ -9,7 +9,7 @@
 // all rescaled by the same online factor; after the last key tile
 //   O = O / l,  mu = r / l,  tO = T / l - mu O,  LSE = ln l + m,  tLSE = mu.
 //
-// Design (sm_100a, one CTA per query tile, 6 warps):
+// Design (sm_100a, one CTA per query tile, 10 warps):
 //   warp 0      TMA producer: Q, tQ once; then K|tK and V|tV tiles of 64 keys
 //               through 3- and 2-deep shared-memory rings (128-byte swizzle).
 //   warp 1      tcgen05 MMA issuer (one thread), also owns the TMEM allocation:
@@ -19,13 +19,18 @@
 //                 T += (P o tS) V                   (A = P o tS from TMEM, N=D)
 //               S/tS are double-buffered in TMEM so the scores of tile j+1 are
 //               computed while tile j's softmax runs.
-//   warps 2-5   softmax / epilogue, one thread per query row: TMEM -> registers,
-//               mask (only where a tile is not entirely visible to the row),
-//               exp2-domain online softmax with a lazily updated max, bf16 P and
-//               P o tS written back over the scores in TMEM, and the final
-//               normalisation and JVP epilogue.
+//   warps 2-9   softmax / epilogue: two warpgroups, each thread owns one query
+//               row and one 32-key half of every key tile (warpgroup g takes
+//               keys [32g, 32g+32)). TMEM -> registers, mask (only where the half
+//               tile is not entirely visible to the row), exp2-domain online
+//               softmax with a lazily updated max shared by the two halves
+//               through shared memory, bf16 P and P o tS written back into the
+//               score columns in TMEM, and the final normalisation and JVP
+//               epilogue (warpgroup g writes output columns [gD/2, (g+1)D/2)).
 // TMEM (512 columns x 128 lanes, fp32): O [0,D) | T [D,2D) | S/tS buffer 0 |
-// S/tS buffer 1, each buffer S [64 cols] then tS [64 cols].
+// S/tS buffer 1, each buffer S [64 cols] then tS [64 cols]. The bf16 P of keys
+// [32g, 32g+32) is packed into S columns [32g, 32g+16) and P o tS into the same
+// columns of tS, so each thread only overwrites score columns it has read.
 //
 // Every wait on an mbarrier is bounded by a time limit; on expiry the kernel
 // records an error code in a device word, drains its own in-flight copies and
@@ -48,7 +53,8 @@ using namespace ptx;
 
 constexpr int BM = kBlockM;  // query rows per tile
 constexpr int BN = kBlockN;  // keys per tile
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale once the max grew by 2^8
 
 template <int D>
@@ -68,10 +74,13 @@ struct Cfg {
   static constexpr int OFF_V = OFF_KT + KS * KT_STAGE;
   static constexpr int OFF_BAR = OFF_V + VS * V_STAGE;
   // barriers: q_full, kv_full[KS], kv_empty[KS], v_full[VS], v_empty[VS],
-  //           s_full[2], p_full[2], o_done[2], drain
-  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 7;
+  //           s_full[2], p_full[2], o_done[2], drain,
+  //           pair[4 lane quarters][2 slots], pair_end[4 lane quarters]
+  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 7 + 12;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  // row-max exchange between the two softmax warpgroups: [2 slots][2 halves][BM] fp32
+  static constexpr int OFF_XCH = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_XCH + 2 * 2 * BM * 4;
   // tensor memory columns
   static constexpr uint32_t COL_O = 0;
   static constexpr uint32_t COL_T = D;
@@ -86,7 +95,7 @@ struct Cfg {
 };
 
 struct Barriers {
-  uint32_t q_full, kv_full, kv_empty, v_full, v_empty, s_full, p_full, o_done, drain;
+  uint32_t q_full, kv_full, kv_empty, v_full, v_empty, s_full, p_full, o_done, drain, pair, pair_end;
 };
 
 template <int D>
@@ -102,6 +111,8 @@ __device__ __forceinline__ Barriers make_barriers(uint32_t base) {
   b.p_full = b.s_full + 16;
   b.o_done = b.p_full + 16;
   b.drain = b.o_done + 16;
+  b.pair = b.drain + 8;
+  b.pair_end = b.pair + 64;
   return b;
 }
 
@@ -148,23 +159,43 @@ __device__ __forceinline__ int32_t tile_at(int32_t j, int32_t t0, int32_t n0, in
   return j < n0 ? t0 + j : t2 + (j - n0);
 }
 
+// Rendezvous of the two softmax warps that share a lane quarter, through an
+// mbarrier with two arrivals (bounded, unlike a named barrier, so an aborting
+// CTA cannot strand the partner). Orders the warps' shared-memory writes and
+// tcgen05 accesses before the partner's subsequent ones.
+__device__ __forceinline__ bool pair_sync(uint32_t mbar, uint32_t parity, int lane,
+                                          volatile int *abort_flag, uint64_t timeout_ns,
+                                          uint32_t site) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(mbar);
+  const bool got = wait_bounded(mbar, parity, abort_flag, timeout_ns, site);
+  tc_fence_after();
+  return __all_sync(0xffffffffu, got);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {
   using C = Cfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint8_t *sgen = smem_raw + (sbase - raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  // 128-byte-swizzled tiles need a 1 KiB aligned base; refuse to run otherwise.
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(&g_device_error, 0u, uint32_t(kErrSmemMisaligned));
+    return;
+  }
+  uint8_t *sgen = smem_raw;
   const Barriers bar = make_barriers<D>(sbase + C::OFF_BAR);
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sgen + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + C::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Work item: heaviest query tiles first, heads fastest.
-  const int32_t qt = p.qtile_order[blockIdx.x / p.BH];
-  const int32_t bh = blockIdx.x % p.BH;
+  // Work item: head by head (its K/V stay in L2 while its tiles run), and
+  // inside a head the heaviest query tiles first.
+  const int32_t bh = blockIdx.x / p.n_qtiles;
+  const int32_t qt = p.qtile_order[blockIdx.x % p.n_qtiles];
   const int32_t q0 = qt * BM;
   const int32_t q1 = min(q0 + BM, p.geom.N);
   int32_t t0, t1, t2, t3;
@@ -183,10 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar.s_full + 8 * b, 1);
-      mbar_init(bar.p_full + 8 * b, 4);  // one arrival per softmax warp
+      mbar_init(bar.p_full + 8 * b, kSoftmaxWarps);  // one arrival per softmax warp
       mbar_init(bar.o_done + 8 * b, 1);
     }
     mbar_init(bar.drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar.pair + 8 * i, 2);  // the two warps of a lane quarter
+    for (int i = 0; i < 4; ++i) mbar_init(bar.pair_end + 8 * i, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -301,8 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < BN / 16; ++kk) {
           // MN-major B: 64-element column blocks C::VBLK apart, 8-key groups 1 KiB apart.
           const uint64_t b_v = sdesc_sw128(vt + kk * 16 * 128, C::VBLK, 1024);
-          mma_ts(tmem + C::COL_O, aP + kk * 8, b_v, ID_OT, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tmem + C::COL_T, aP + BN + kk * 8, b_v, ID_T, 1u);
+          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;  // packed P columns of keys 16kk..
+          mma_ts(tmem + C::COL_O, aP + pc, b_v, ID_OT, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::COL_T, aP + BN + pc, b_v, ID_T, 1u);
         }
         tc_commit(bar.v_empty + 8 * s);
         tc_commit(bar.o_done + 8 * (i & 1));
@@ -318,10 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------- softmax + epilogue
+    const int g = (warp - 2) >> 2;            // key half of each tile owned by this warpgroup
     const int sub = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = sub * 32 + lane;          // query row within the tile
     const int32_t q = q0 + row;
     const uint32_t lane_addr = tmem + (uint32_t(sub * 32) << 16);
+    float *xch = reinterpret_cast<float *>(sgen + C::OFF_XCH);  // [slot][half][row]
     int32_t a0, b0, a1, b1;
     if (q < p.geom.N) {
       row_key_ranges(p.geom, q, a0, b0, a1, b1);
@@ -333,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2e;
     const float scale = p.scale;
     float m_run = -INFINITY;  // running max of s * scale * log2(e), possibly stale by < 2^8
-    float l_run = 0.f, r_run = 0.f;
+    float l_run = 0.f, r_run = 0.f;  // partial sums over this thread's key halves
     bool ok = true;
 
     for (int32_t j = 0; j < ntiles; ++j) {
@@ -344,37 +380,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int32_t k0 = tile_at(j, t0, n0, t2) * BN;
-      const uint32_t cS = lane_addr + C::COL_S0 + b * C::BUF_COLS;
-      float s[BN];
-      {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(cS, r0);
-        tmem_ld32(cS + 32, r1);
+      const int32_t kh = tile_at(j, t0, n0, t2) * BN + 32 * g;  // first key of this half
+      const uint32_t cS = lane_addr + C::COL_S0 + b * C::BUF_COLS + 32 * g;
+      const uint32_t cT = cS + BN;
+      uint32_t rs[32], rt[32];
+      tmem_ld32x2(cS, cT, rs, rt);
+      float s[32], t[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        s[i] = __uint_as_float(rs[i]);
+        t[i] = __uint_as_float(rt[i]) * scale;
+      }
+      // Mask only where this half tile is not entirely inside the row's ranges.
+      const bool full = (kh >= a0 && kh + 32 <= b0) || (kh >= a1 && kh + 32 <= b1);
+      if (!full) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(r0[i]);
-          s[32 + i] = __uint_as_float(r1[i]);
-        }
-      }
-      // Mask only where this tile is not entirely inside the row's key ranges.
-      const bool full = (k0 >= a0 && k0 + BN <= b0) || (k0 >= a1 && k0 + BN <= b1);
-      uint32_t vis_lo = 0xffffffffu, vis_hi = 0xffffffffu;
-      if (!full) {
-        vis_lo = vis_hi = 0;
-#pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          const int32_t key = k0 + i;
+          const int32_t key = kh + i;
           const bool v = (key >= a0 && key < b0) || (key >= a1 && key < b1);
-          if (i < 32) vis_lo |= uint32_t(v) << i;
-          else vis_hi |= uint32_t(v) << (i - 32);
           s[i] = v ? s[i] : -INFINITY;
+          t[i] = v ? t[i] : 0.f;
         }
       }
-      float tmax = s[0];
+      float mx[8];
 #pragma unroll
-      for (int i = 1; i < BN; ++i) tmax = fmaxf(tmax, s[i]);
-      const float m_tile = tmax * sl2;  // -inf if the row sees nothing here
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
+      const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      // Exchange the half-row max with the other warpgroup. The barrier also
+      // orders both threads' score reads before either writes P into TMEM.
+      xch[(b * 2 + g) * BM + row] = hmax;
+      if (!pair_sync(bar.pair + 8 * (sub * 2 + b), (j >> 1) & 1, lane, abort_flag, p.timeout_ns,
+                     10)) {
+        ok = false;
+        break;
+      }
+      const float tmax = fmaxf(hmax, xch[(b * 2 + (g ^ 1)) * BM + row]);
+      const float m_tile = tmax * sl2;  // -inf if the row sees nothing in this tile
       // Lazy rescale: keep the old max unless the new one exceeds it by 2^8.
       const bool grow = m_tile > m_run + kRescaleThreshold;
       const bool had_acc = m_run != -INFINITY;  // accumulators hold non-zero data
@@ -386,8 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_tile;
       }
       if (__any_sync(0xffffffffu, grow && had_acc) && j > 0) {
-        // O and T of this warp's rows must be scaled by alpha; wait until the
-        // value MMAs of the previous tile have landed.
+        // This warpgroup's accumulator (O for g=0, T for g=1) must be scaled by
+        // alpha once the value MMAs of the previous tile have landed.
         const int pb = (j - 1) & 1;
         const bool g2 =
             wait_bounded(bar.o_done + 8 * pb, ((j - 1) >> 1) & 1, abort_flag, p.timeout_ns, 8);
@@ -396,52 +439,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        const uint32_t acc = lane_addr + (g ? C::COL_T : C::COL_O);
 #pragma unroll 1
-        for (int c = 0; c < 2 * D; c += 32) {
+        for (int c = 0; c < D; c += 32) {
           uint32_t r[32];
-          tmem_ld32(lane_addr + C::COL_O + c, r);
+          tmem_ld32(acc + c, r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(lane_addr + C::COL_O + c, r);
+          tmem_st32(acc + c, r);
         }
-        tmem_wait_st();
       }
       const float ref = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(s*scale*log2e - ref), rounded to bf16 and written over S.
-      float lsum = 0.f;
+      // P = 2^(s*scale*log2e - ref) and P o tS, rounded to bf16 and packed into
+      // this half's first 16 score columns.
+      float ls[4] = {0.f, 0.f, 0.f, 0.f}, rsum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[16], tk[16];
 #pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        s[i] = ex2(fmaf(s[i], sl2, -ref));
-        lsum += s[i];
+      for (int i = 0; i < 16; ++i) {
+        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+        const float qa = pa * t[2 * i], qb = pb * t[2 * i + 1];
+        ls[i & 3] += pa + pb;
+        rsum[i & 3] += qa + qb;
+        pk[i] = pack_bf16(pa, pb);
+        tk[i] = pack_bf16(qa, qb);
       }
-      l_run += lsum;
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(s[2 * i], s[2 * i + 1]);
-        tmem_st32(cS, pk);
-      }
-      // P o tS (scaled), rounded to bf16 and written over tS; r += sum p ts.
-      float rsum = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t tr[32];
-        tmem_ld32(cS + BN + 32 * h, tr);
-        const uint32_t vis = h ? vis_hi : vis_lo;
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float ta = __uint_as_float(tr[2 * i]) * scale;
-          float tb = __uint_as_float(tr[2 * i + 1]) * scale;
-          ta = ((vis >> (2 * i)) & 1u) ? ta : 0.f;
-          tb = ((vis >> (2 * i + 1)) & 1u) ? tb : 0.f;
-          const float pa = s[32 * h + 2 * i] * ta, pb = s[32 * h + 2 * i + 1] * tb;
-          rsum += pa + pb;
-          pk[i] = pack_bf16(pa, pb);
-        }
-        tmem_st16(cS + BN + 16 * h, pk);
-      }
-      r_run += rsum;
+      tmem_st16(cS, pk);
+      tmem_st16(cT, tk);
+      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      r_run += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -449,22 +475,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (ok && ntiles > 0) {
+      // Combine the two halves' partial sums (both relative to the same max).
+      // Slot ntiles&1 was last read at tile ntiles-2, before the partner's
+      // final pair rendezvous; slot (ntiles-1)&1 is free once the first
+      // rendezvous below has passed.
+      const int s0 = ntiles & 1, s1 = s0 ^ 1;
+      xch[(s0 * 2 + g) * BM + row] = l_run;
+      bool got = pair_sync(bar.pair_end + 8 * sub, 0, lane, abort_flag, p.timeout_ns, 11);
+      const float l_tot = l_run + xch[(s0 * 2 + (g ^ 1)) * BM + row];
+      if (got) {
+        xch[(s1 * 2 + g) * BM + row] = r_run;
+        got = pair_sync(bar.pair_end + 8 * sub, 1, lane, abort_flag, p.timeout_ns, 11);
+      }
+      const float r_tot = r_run + xch[(s1 * 2 + (g ^ 1)) * BM + row];
       const int32_t last = ntiles - 1;
-      const bool got =
-          wait_bounded(bar.o_done + 8 * (last & 1), (last >> 1) & 1, abort_flag, p.timeout_ns, 9);
+      if (got)
+        got = wait_bounded(bar.o_done + 8 * (last & 1), (last >> 1) & 1, abort_flag, p.timeout_ns, 9);
       if (__all_sync(0xffffffffu, got)) {
         tc_fence_after();
-        const float inv_l = 1.f / l_run;
-        const float mu = r_run * inv_l;
+        const float inv_l = 1.f / l_tot;
+        const float mu = r_tot * inv_l;
         const bool store = q < p.geom.N;
         const size_t rowoff = (size_t(bh) * p.geom.N + (store ? q : 0)) * D;
         uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
         uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
           uint32_t ro[32], rt[32];
-          tmem_ld32(lane_addr + C::COL_O + c, ro);
-          tmem_ld32(lane_addr + C::COL_T + c, rt);
+          tmem_ld32x2(lane_addr + C::COL_O + c, lane_addr + C::COL_T + c, ro, rt);
           uint32_t po[16], pt[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -483,9 +521,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (store) {
+        if (store && g == 0) {
           const size_t ri = size_t(bh) * p.geom.N + q;
-          p.lse[ri] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+          p.lse[ri] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
           p.tlse[ri] = mu;
         }
       }

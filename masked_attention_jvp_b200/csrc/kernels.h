@@ -19,7 +19,8 @@ constexpr int kMaxQTiles = 4096;
 // Device error word values (first error wins). Low byte: where a wait gave up.
 enum DeviceError : uint32_t {
   kErrNone = 0,
-  kErrTimeoutBase = 0x100,  // | wait site
+  kErrTimeoutBase = 0x100,     // | wait site
+  kErrSmemMisaligned = 0x200,  // dynamic shared memory not 1 KiB aligned
 };
 
 struct Sm100Params {
