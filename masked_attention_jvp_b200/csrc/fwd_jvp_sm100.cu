@@ -161,16 +161,14 @@ __device__ __forceinline__ int32_t tile_at(int32_t j, int32_t t0, int32_t n0, in
 
 // Rendezvous of the two softmax warps that share a lane quarter, through an
 // mbarrier with two arrivals (bounded, unlike a named barrier, so an aborting
-// CTA cannot strand the partner). Orders the warps' shared-memory writes and
-// tcgen05 accesses before the partner's subsequent ones.
+// CTA cannot strand the partner). Orders each warp's shared-memory writes
+// before the partner's subsequent reads (arrive releases, the wait acquires).
 __device__ __forceinline__ bool pair_sync(uint32_t mbar, uint32_t parity, int lane,
                                           volatile int *abort_flag, uint64_t timeout_ns,
                                           uint32_t site) {
-  tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(mbar);
   const bool got = wait_bounded(mbar, parity, abort_flag, timeout_ns, site);
-  tc_fence_after();
   return __all_sync(0xffffffffu, got);
 }
 
@@ -299,47 +297,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t ID_TS = idesc_bf16_f32(BM, BN, 0);      // tQ K^T
       constexpr uint32_t ID_OT = idesc_bf16_f32(BM, 2 * D, 1);   // P [V|tV]
       constexpr uint32_t ID_T = idesc_bf16_f32(BM, D, 1);        // (P o tS) V
-      const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
+      // Operand descriptors: one base per buffer, then compile-time byte offsets
+      // (added to the start-address field, which cannot carry out of its 14 bits
+      // for shared-memory addresses below 256 KiB).
+      const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
+      const uint64_t dTQ = sdesc_sw128(sbase + C::OFF_TQ, 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_KT, 16, 1024);
+      // MN-major B: 64-element column blocks C::VBLK apart, 8-key groups 1 KiB apart.
+      const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::VBLK, 1024);
+      const uint32_t tS0 = tmem + C::COL_S0;
       bool ok = wait_bounded(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
+      int ks = 0, kph = 0, vs = 0, vph = 0;  // ring slots and phase parities
       auto issue_scores = [&](int32_t j) -> bool {
-        const int s = j % C::KS;
-        if (!wait_bounded(bar.kv_full + 8 * s, (j / C::KS) & 1, abort_flag, p.timeout_ns, 4))
-          return false;
+        if (!wait_bounded(bar.kv_full + 8 * ks, kph, abort_flag, p.timeout_ns, 4)) return false;
         tc_fence_after();
-        const uint32_t kt = sbase + C::OFF_KT + s * C::KT_STAGE;
-        const uint32_t dS = tmem + C::COL_S0 + (j & 1) * C::BUF_COLS;
+        const uint64_t dK = dK0 + uint64_t((ks * C::KT_STAGE) >> 4);
+        const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
-          const uint64_t a_q = sdesc_sw128(sq + (kk >> 2) * C::QBLK + koff, 16, 1024);
-          const uint64_t a_tq = sdesc_sw128(stq + (kk >> 2) * C::QBLK + koff, 16, 1024);
-          const uint64_t b_k = sdesc_sw128(kt + (kk >> 2) * C::KBLK + koff, 16, 1024);
-          mma_ss(dS, a_q, b_k, ID_S, kk > 0 ? 1u : 0u);
-          mma_ss(dS + BN, a_tq, b_k, ID_TS, 1u);
+          // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
+          const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
+          const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
+          mma_ss(dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
+          mma_ss(dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
         }
-        tc_commit(bar.kv_empty + 8 * s);
+        tc_commit(bar.kv_empty + 8 * ks);
         tc_commit(bar.s_full + 8 * (j & 1));
+        if (++ks == C::KS) { ks = 0; kph ^= 1; }
         return true;
       };
       auto issue_values = [&](int32_t i) -> bool {
-        const int s = i % C::VS;
         if (!wait_bounded(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5))
           return false;
-        if (!wait_bounded(bar.v_full + 8 * s, (i / C::VS) & 1, abort_flag, p.timeout_ns, 6))
-          return false;
+        if (!wait_bounded(bar.v_full + 8 * vs, vph, abort_flag, p.timeout_ns, 6)) return false;
         tc_fence_after();
-        const uint32_t vt = sbase + C::OFF_V + s * C::V_STAGE;
-        const uint32_t aP = tmem + C::COL_S0 + (i & 1) * C::BUF_COLS;
+        const uint64_t dV = dV0 + uint64_t((vs * C::V_STAGE) >> 4);
+        const uint32_t aP = tS0 + (i & 1) * C::BUF_COLS;
+        const uint32_t first = i > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // MN-major B: 64-element column blocks C::VBLK apart, 8-key groups 1 KiB apart.
-          const uint64_t b_v = sdesc_sw128(vt + kk * 16 * 128, C::VBLK, 1024);
-          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;  // packed P columns of keys 16kk..
-          mma_ts(tmem + C::COL_O, aP + pc, b_v, ID_OT, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tmem + C::COL_T, aP + BN + pc, b_v, ID_T, 1u);
+          const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
+          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
+          mma_ts(tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
+          mma_ts(tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
         }
-        tc_commit(bar.v_empty + 8 * s);
+        tc_commit(bar.v_empty + 8 * vs);
         tc_commit(bar.o_done + 8 * (i & 1));
+        if (++vs == C::VS) { vs = 0; vph ^= 1; }
         return true;
       };
       for (int32_t j = 0; ok && j <= ntiles; ++j) {
@@ -385,21 +389,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t cT = cS + BN;
       uint32_t rs[32], rt[32];
       tmem_ld32x2(cS, cT, rs, rt);
-      float s[32], t[32];
+      float s[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        s[i] = __uint_as_float(rs[i]);
-        t[i] = __uint_as_float(rt[i]) * scale;
-      }
+      for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(rs[i]);
       // Mask only where this half tile is not entirely inside the row's ranges.
       const bool full = (kh >= a0 && kh + 32 <= b0) || (kh >= a1 && kh + 32 <= b1);
+      uint32_t vis = 0xffffffffu;
       if (!full) {
+        vis = 0;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int32_t key = kh + i;
           const bool v = (key >= a0 && key < b0) || (key >= a1 && key < b1);
+          vis |= uint32_t(v) << i;
           s[i] = v ? s[i] : -INFINITY;
-          t[i] = v ? t[i] : 0.f;
         }
       }
       float mx[8];
@@ -408,8 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
       const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      // Exchange the half-row max with the other warpgroup. The barrier also
-      // orders both threads' score reads before either writes P into TMEM.
+      // Exchange the half-row max with the other warpgroup.
       xch[(b * 2 + g) * BM + row] = hmax;
       if (!pair_sync(bar.pair + 8 * (sub * 2 + b), (j >> 1) & 1, lane, abort_flag, p.timeout_ns,
                      10)) {
@@ -454,15 +456,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this half's first 16 score columns.
       float ls[4] = {0.f, 0.f, 0.f, 0.f}, rsum[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[16], tk[16];
+      if (full) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-        const float qa = pa * t[2 * i], qb = pb * t[2 * i + 1];
-        ls[i & 3] += pa + pb;
-        rsum[i & 3] += qa + qb;
-        pk[i] = pack_bf16(pa, pb);
-        tk[i] = pack_bf16(qa, qb);
+        for (int i = 0; i < 16; ++i) {
+          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+          const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
+          const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
+          ls[i & 3] += pa + pb;
+          rsum[i & 3] += qa + qb;
+          pk[i] = pack_bf16(pa, pb);
+          tk[i] = pack_bf16(qa, qb);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+          // invisible keys carry no tangent: select rather than multiply, so a
+          // non-finite score tangent of a masked key cannot leak in as 0 * inf
+          const float ta = ((vis >> (2 * i)) & 1u) ? __uint_as_float(rt[2 * i]) * scale : 0.f;
+          const float tb = ((vis >> (2 * i + 1)) & 1u) ? __uint_as_float(rt[2 * i + 1]) * scale : 0.f;
+          const float qa = pa * ta, qb = pb * tb;
+          ls[i & 3] += pa + pb;
+          rsum[i & 3] += qa + qb;
+          pk[i] = pack_bf16(pa, pb);
+          tk[i] = pack_bf16(qa, qb);
+        }
       }
       tmem_st16(cS, pk);
       tmem_st16(cT, tk);
