@@ -153,6 +153,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ------------------------------------------------------------- multi-rank
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Slowest rank's time: an all-reduce MAX of one scalar (the only
+    collective of the benchmark; none sits on the data path)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: int, world: int, steps: int, slowest_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own copy of the workload
+    (weak scaling), all of them within the slowest rank's time."""
+    return world * flops_per_rank * steps / (slowest_ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU arm
 def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
     """Same metric through the public API from pinned host buffers: every step
@@ -172,12 +189,8 @@ def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
         caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(world * fl * steps / (ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(whole_job_tflops(fl, world, steps, ms), 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 
@@ -221,13 +234,9 @@ def bench_gpu(args, rank, world, local_rank):
     barrier()
     caj.device_status()
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * fl * args.steps / (total_ms / 1e3) / 1e12
+    value = whole_job_tflops(fl, world, args.steps, total_ms)
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -248,6 +257,7 @@ def bench_gpu(args, rank, world, local_rank):
         "config": workload_config(w, {"parallelism": f"replica x{world}" if world > 1 else "single GPU"}),
         "pct_of_dense_bf16_peak": round(100.0 * value / world / DENSE_BF16_SPEC_TFLOPS, 2),
         "ms_per_step_min": round(min(per), 4), "ms_per_step_median": round(statistics.median(per), 4),
+        "ms_per_step_each": [round(x, 3) for x in per],
         "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": args.steps,

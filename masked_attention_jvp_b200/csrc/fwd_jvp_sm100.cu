@@ -10,8 +10,11 @@
 //   O = O / l,  mu = r / l,  tO = T / l - mu O,  LSE = ln l + m,  tLSE = mu.
 //
 // Design (sm_100a, one CTA per query tile, 10 warps):
-//   warp 0      TMA producer: Q, tQ once; then K|tK and V|tV tiles of 64 keys
-//               through 3- and 2-deep shared-memory rings (128-byte swizzle).
+//   warp 0      TMA producer: Q, tQ once; then, per step j, the K|tK tile of
+//               key tile j and the V|tV tile of key tile j-1, both completing on
+//               one barrier, through 2-deep shared-memory rings (128-byte swizzle).
+//               K stage j%2 is released by the score-MMA commit of tile j, V stage
+//               j%2 by the value-MMA commit of tile j.
 //   warp 1      tcgen05 MMA issuer (one thread), also owns the TMEM allocation:
 //                 [S | tS_1] = Q [K ; tK]^T        (one N=128 MMA per k-step)
 //                 tS += tQ K^T                      (N=64)
@@ -66,17 +69,17 @@ struct Cfg {
   static constexpr int KT_STAGE = NB * KBLK;
   static constexpr int VBLK = BN * 128;                // one column block of V (or tV)
   static constexpr int V_STAGE = 2 * NB * VBLK;        // V blocks, then tV blocks
-  static constexpr int KS = (D == 128) ? 3 : 4;
-  static constexpr int VS = (D == 128) ? 2 : 4;
+  // K stage j%2 is released by s_full[j%2], V stage j%2 by o_done[j%2]
+  static constexpr int KS = 2;
+  static constexpr int VS = 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_TQ = Q_BYTES;
   static constexpr int OFF_KT = 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_KT + KS * KT_STAGE;
   static constexpr int OFF_BAR = OFF_V + VS * V_STAGE;
-  // barriers: q_full, kv_full[KS], kv_empty[KS], v_full[VS], v_empty[VS],
-  //           s_full[2], p_full[2], o_done[2], drain,
+  // barriers: q_full, x_full[2], s_full[2], p_full[2], o_done[2], drain,
   //           pair[4 lane quarters][2 slots], pair_end[4 lane quarters]
-  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 7 + 12;
+  static constexpr int NBAR = 1 + 2 + 7 + 12;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
   // row-max exchange between the two softmax warpgroups: [2 slots][2 halves][BM] fp32
   static constexpr int OFF_XCH = OFF_MISC + 16;
@@ -92,10 +95,11 @@ struct Cfg {
   static constexpr uint32_t Q_TX = 2 * Q_BYTES;
   static constexpr uint32_t KT_TX = KT_STAGE;
   static constexpr uint32_t V_TX = V_STAGE;
+  static_assert(KT_TX + V_TX < (1u << 20), "transaction count limit");
 };
 
 struct Barriers {
-  uint32_t q_full, kv_full, kv_empty, v_full, v_empty, s_full, p_full, o_done, drain, pair, pair_end;
+  uint32_t q_full, x_full, s_full, p_full, o_done, drain, pair, pair_end;
 };
 
 template <int D>
@@ -103,11 +107,8 @@ __device__ __forceinline__ Barriers make_barriers(uint32_t base) {
   using C = Cfg<D>;
   Barriers b;
   b.q_full = base;
-  b.kv_full = base + 8;
-  b.kv_empty = b.kv_full + 8 * C::KS;
-  b.v_full = b.kv_empty + 8 * C::KS;
-  b.v_empty = b.v_full + 8 * C::VS;
-  b.s_full = b.v_empty + 8 * C::VS;
+  b.x_full = base + 8;
+  b.s_full = b.x_full + 16;
   b.p_full = b.s_full + 16;
   b.o_done = b.p_full + 16;
   b.drain = b.o_done + 16;
@@ -127,7 +128,7 @@ __device__ __noinline__ void raise_error(volatile int *abort_flag, uint32_t code
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile int *abort_flag, uint64_t timeout_ns,
                                              uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1; it < 0x40000000u; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -202,15 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q_full, 1);
-    for (int s = 0; s < C::KS; ++s) {
-      mbar_init(bar.kv_full + 8 * s, 1);
-      mbar_init(bar.kv_empty + 8 * s, 1);
-    }
-    for (int s = 0; s < C::VS; ++s) {
-      mbar_init(bar.v_full + 8 * s, 1);
-      mbar_init(bar.v_empty + 8 * s, 1);
-    }
     for (int b = 0; b < 2; ++b) {
+      mbar_init(bar.x_full + 8 * b, 1);
       mbar_init(bar.s_full + 8 * b, 1);
       mbar_init(bar.p_full + 8 * b, kSoftmaxWarps);  // one arrival per softmax warp
       mbar_init(bar.o_done + 8 * b, 1);
@@ -242,53 +236,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
         tma_load_3d(stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
       }
-      int32_t k_issued = 0, v_issued = 0;
-      bool ok = true;
-      auto issue_k = [&](int32_t j) -> bool {
-        const int s = j % C::KS;
-        if (j >= C::KS &&
-            !wait_bounded(bar.kv_empty + 8 * s, ((j / C::KS) - 1) & 1, abort_flag, p.timeout_ns, 1))
-          return false;
-        const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
-        const uint32_t dst = sbase + C::OFF_KT + s * C::KT_STAGE;
-        const uint32_t fb = bar.kv_full + 8 * s;
-        mbar_arrive_expect_tx(fb, C::KT_TX);
-        for (int c = 0; c < C::NB; ++c) {
-          tma_load_3d(dst + c * C::KBLK, &p.tm_k, fb, c * 64, key0, bh);
-          tma_load_3d(dst + c * C::KBLK + BN * 128, &p.tm_tk, fb, c * 64, key0, bh);
+      // Step j loads K|tK of key tile j (j < ntiles) into K stage j%2 and V|tV
+      // of key tile j-1 (j >= 1) into V stage (j-1)%2, completing on x_full[j%2].
+      int32_t steps_armed = 0;
+      for (int32_t j = 0; j <= ntiles; ++j) {
+        const int b = j & 1;
+        // S(j-2) done: K stage b and x_full[b]'s previous phase are consumed
+        if (j >= 2 &&
+            !wait_bounded(bar.s_full + 8 * b, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 1))
+          break;
+        // OT(j-3) done: V stage (j-1)%2 is free
+        if (j >= 3 && !wait_bounded(bar.o_done + 8 * ((j - 1) & 1), (((j - 1) >> 1) - 1) & 1,
+                                    abort_flag, p.timeout_ns, 2))
+          break;
+        const bool has_k = j < ntiles, has_v = j >= 1;
+        const uint32_t fb = bar.x_full + 8 * b;
+        mbar_arrive_expect_tx(fb, (has_k ? C::KT_TX : 0u) + (has_v ? C::V_TX : 0u));
+        if (has_k) {
+          const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
+          const uint32_t dst = sbase + C::OFF_KT + b * C::KT_STAGE;
+          for (int c = 0; c < C::NB; ++c) {
+            tma_load_3d(dst + c * C::KBLK, &p.tm_k, fb, c * 64, key0, bh);
+            tma_load_3d(dst + c * C::KBLK + BN * 128, &p.tm_tk, fb, c * 64, key0, bh);
+          }
         }
-        k_issued = j + 1;
-        return true;
-      };
-      auto issue_v = [&](int32_t j) -> bool {
-        const int s = j % C::VS;
-        if (j >= C::VS &&
-            !wait_bounded(bar.v_empty + 8 * s, ((j / C::VS) - 1) & 1, abort_flag, p.timeout_ns, 2))
-          return false;
-        const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
-        const uint32_t dst = sbase + C::OFF_V + s * C::V_STAGE;
-        const uint32_t fb = bar.v_full + 8 * s;
-        mbar_arrive_expect_tx(fb, C::V_TX);
-        for (int c = 0; c < C::NB; ++c) {
-          tma_load_3d(dst + c * C::VBLK, &p.tm_v, fb, c * 64, key0, bh);
-          tma_load_3d(dst + (C::NB + c) * C::VBLK, &p.tm_tv, fb, c * 64, key0, bh);
+        if (has_v) {
+          const int32_t key0 = tile_at(j - 1, t0, n0, t2) * BN;
+          const uint32_t dst = sbase + C::OFF_V + ((j - 1) & 1) * C::V_STAGE;
+          for (int c = 0; c < C::NB; ++c) {
+            tma_load_3d(dst + c * C::VBLK, &p.tm_v, fb, c * 64, key0, bh);
+            tma_load_3d(dst + (C::NB + c) * C::VBLK, &p.tm_tv, fb, c * 64, key0, bh);
+          }
         }
-        v_issued = j + 1;
-        return true;
-      };
-      // K runs one tile ahead of V: the scores of tile j+1 are needed before
-      // the value products of tile j.
-      ok = issue_k(0);
-      for (int32_t j = 0; ok && j < ntiles; ++j) {
-        if (j + 1 < ntiles) ok = issue_k(j + 1);
-        if (ok) ok = issue_v(j);
+        steps_armed = j + 1;
       }
       // Drain: every copy this thread issued must land before the CTA exits.
       drain_wait(bar.q_full, 0, p.timeout_ns);
-      for (int32_t j = (k_issued > C::KS ? k_issued - C::KS : 0); j < k_issued; ++j)
-        drain_wait(bar.kv_full + 8 * (j % C::KS), (j / C::KS) & 1, p.timeout_ns);
-      for (int32_t j = (v_issued > C::VS ? v_issued - C::VS : 0); j < v_issued; ++j)
-        drain_wait(bar.v_full + 8 * (j % C::VS), (j / C::VS) & 1, p.timeout_ns);
+      for (int32_t j = (steps_armed > 2 ? steps_armed - 2 : 0); j < steps_armed; ++j)
+        drain_wait(bar.x_full + 8 * (j & 1), (j >> 1) & 1, p.timeout_ns);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -307,48 +292,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::VBLK, 1024);
       const uint32_t tS0 = tmem + C::COL_S0;
       bool ok = wait_bounded(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
-      int ks = 0, kph = 0, vs = 0, vph = 0;  // ring slots and phase parities
-      auto issue_scores = [&](int32_t j) -> bool {
-        if (!wait_bounded(bar.kv_full + 8 * ks, kph, abort_flag, p.timeout_ns, 4)) return false;
-        tc_fence_after();
-        const uint64_t dK = dK0 + uint64_t((ks * C::KT_STAGE) >> 4);
-        const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
-          const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
-          const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
-          mma_ss(dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
-          mma_ss(dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
-        }
-        tc_commit(bar.kv_empty + 8 * ks);
-        tc_commit(bar.s_full + 8 * (j & 1));
-        if (++ks == C::KS) { ks = 0; kph ^= 1; }
-        return true;
-      };
-      auto issue_values = [&](int32_t i) -> bool {
-        if (!wait_bounded(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5))
-          return false;
-        if (!wait_bounded(bar.v_full + 8 * vs, vph, abort_flag, p.timeout_ns, 6)) return false;
-        tc_fence_after();
-        const uint64_t dV = dV0 + uint64_t((vs * C::V_STAGE) >> 4);
-        const uint32_t aP = tS0 + (i & 1) * C::BUF_COLS;
-        const uint32_t first = i > 0 ? 1u : 0u;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
-          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
-          mma_ts(tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
-          mma_ts(tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
-        }
-        tc_commit(bar.v_empty + 8 * vs);
-        tc_commit(bar.o_done + 8 * (i & 1));
-        if (++vs == C::VS) { vs = 0; vph ^= 1; }
-        return true;
-      };
+      // Step j: scores of key tile j, then value products of key tile j-1. One
+      // probe covers K(j) and V(j-1); a second one waits for P(j-1).
       for (int32_t j = 0; ok && j <= ntiles; ++j) {
-        if (j < ntiles) ok = issue_scores(j);
-        if (ok && j >= 1) ok = issue_values(j - 1);
+        if (!wait_bounded(bar.x_full + 8 * (j & 1), (j >> 1) & 1, abort_flag, p.timeout_ns, 4)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (j < ntiles) {
+          const uint64_t dK = dK0 + uint64_t(((j & 1) * C::KT_STAGE) >> 4);
+          const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
+            const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
+            const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
+            mma_ss(dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
+            mma_ss(dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
+          }
+          tc_commit(bar.s_full + 8 * (j & 1));
+        }
+        if (j >= 1) {
+          const int32_t i = j - 1;
+          if (!wait_bounded(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dV = dV0 + uint64_t(((i & 1) * C::V_STAGE) >> 4);
+          const uint32_t aP = tS0 + (i & 1) * C::BUF_COLS;
+          const uint32_t first = i > 0 ? 1u : 0u;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
+            const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
+            mma_ts(tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
+            mma_ts(tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
+          }
+          tc_commit(bar.o_done + 8 * (i & 1));
+        }
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       tc_commit(bar.drain);

@@ -1,0 +1,53 @@
+"""Multi-process host path of bench.py on the CPU: two gloo ranks, each timing its
+own copy of the workload, combine the slowest rank's time with one all-reduce MAX
+and report whole-job throughput. No GPU is involved."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        local_ms = [10.0, 12.5][rank]
+        slowest = bench.max_over_ranks(local_ms, world, torch.device("cpu"))
+        value = bench.whole_job_tflops(20_724_000_000_000, world, 4, slowest)
+        q.put((rank, slowest, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    for rank, slowest, value in got:
+        assert slowest == 12.5
+        # 2 ranks x 4 steps x 20.724 TFLOP in 12.5 ms
+        assert value == pytest.approx(2 * 4 * 20.724 / 12.5e-3)
+
+
+def test_single_rank_needs_no_collective():
+    import bench
+    assert bench.max_over_ranks(3.0, 1, torch.device("cpu")) == 3.0
+    assert bench.whole_job_tflops(10**12, 1, 1, 1000.0) == pytest.approx(1.0)
