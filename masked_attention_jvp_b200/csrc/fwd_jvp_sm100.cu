@@ -155,6 +155,14 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// Bits [lo, hi) of a 32-bit mask, bounds clamped to [0, 32].
+__device__ __forceinline__ uint32_t range_bits(int32_t lo, int32_t hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 32);
+  if (hi <= lo) return 0u;
+  return uint32_t(((1ull << hi) - 1ull) & ~((1ull << lo) - 1ull));
+}
+
 // Key tile index of the j-th visited tile.
 __device__ __forceinline__ int32_t tile_at(int32_t j, int32_t t0, int32_t n0, int32_t t2) {
   return j < n0 ? t0 + j : t2 + (j - n0);
@@ -171,6 +179,12 @@ __device__ __forceinline__ bool pair_sync(uint32_t mbar, uint32_t parity, int la
   if (lane == 0) mbar_arrive(mbar);
   const bool got = wait_bounded(mbar, parity, abort_flag, timeout_ns, site);
   return __all_sync(0xffffffffu, got);
+}
+
+// Bounded wait by a whole warp, with a warp-uniform outcome.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          uint64_t timeout_ns, uint32_t site) {
+  return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, timeout_ns, site));
 }
 
 template <int D>
@@ -226,117 +240,117 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform addresses stay in uniform
+    // registers); one elected lane issues the copies.
+    const uint32_t leader = elect_one();
+    if (leader) {
       prefetch_tmap(&p.tm_q);
       prefetch_tmap(&p.tm_k);
       prefetch_tmap(&p.tm_v);
-      const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
-      mbar_arrive_expect_tx(bar.q_full, C::Q_TX);
-      for (int c = 0; c < C::NB; ++c) {
-        tma_load_3d(sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
-        tma_load_3d(stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
-      }
-      // Step j loads K|tK of key tile j (j < ntiles) into K stage j%2 and V|tV
-      // of key tile j-1 (j >= 1) into V stage (j-1)%2, completing on x_full[j%2].
-      int32_t steps_armed = 0;
-      for (int32_t j = 0; j <= ntiles; ++j) {
-        const int b = j & 1;
-        // S(j-2) done: K stage b and x_full[b]'s previous phase are consumed
-        if (j >= 2 &&
-            !wait_bounded(bar.s_full + 8 * b, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 1))
-          break;
-        // OT(j-3) done: V stage (j-1)%2 is free
-        if (j >= 3 && !wait_bounded(bar.o_done + 8 * ((j - 1) & 1), (((j - 1) >> 1) - 1) & 1,
-                                    abort_flag, p.timeout_ns, 2))
-          break;
-        const bool has_k = j < ntiles, has_v = j >= 1;
-        const uint32_t fb = bar.x_full + 8 * b;
-        mbar_arrive_expect_tx(fb, (has_k ? C::KT_TX : 0u) + (has_v ? C::V_TX : 0u));
-        if (has_k) {
-          const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
-          const uint32_t dst = sbase + C::OFF_KT + b * C::KT_STAGE;
-          for (int c = 0; c < C::NB; ++c) {
-            tma_load_3d(dst + c * C::KBLK, &p.tm_k, fb, c * 64, key0, bh);
-            tma_load_3d(dst + c * C::KBLK + BN * 128, &p.tm_tk, fb, c * 64, key0, bh);
-          }
-        }
-        if (has_v) {
-          const int32_t key0 = tile_at(j - 1, t0, n0, t2) * BN;
-          const uint32_t dst = sbase + C::OFF_V + ((j - 1) & 1) * C::V_STAGE;
-          for (int c = 0; c < C::NB; ++c) {
-            tma_load_3d(dst + c * C::VBLK, &p.tm_v, fb, c * 64, key0, bh);
-            tma_load_3d(dst + (C::NB + c) * C::VBLK, &p.tm_tv, fb, c * 64, key0, bh);
-          }
-        }
-        steps_armed = j + 1;
-      }
-      // Drain: every copy this thread issued must land before the CTA exits.
-      drain_wait(bar.q_full, 0, p.timeout_ns);
-      for (int32_t j = (steps_armed > 2 ? steps_armed - 2 : 0); j < steps_armed; ++j)
-        drain_wait(bar.x_full + 8 * (j & 1), (j >> 1) & 1, p.timeout_ns);
     }
+    const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
+    mbar_arrive_expect_tx_if(leader, bar.q_full, C::Q_TX);
+    for (int c = 0; c < C::NB; ++c) {
+      tma_load_3d(leader, sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
+      tma_load_3d(leader, stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
+    }
+    // Step j loads K|tK of key tile j (j < ntiles) into K stage j%2 and V|tV
+    // of key tile j-1 (j >= 1) into V stage (j-1)%2, completing on x_full[j%2].
+    int32_t steps_armed = 0;
+    for (int32_t j = 0; j <= ntiles; ++j) {
+      const int b = j & 1;
+      // S(j-2) done: K stage b and x_full[b]'s previous phase are consumed
+      if (j >= 2 && !warp_wait(bar.s_full + 8 * b, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 1))
+        break;
+      // OT(j-3) done: V stage (j-1)%2 is free
+      if (j >= 3 && !warp_wait(bar.o_done + 8 * ((j - 1) & 1), (((j - 1) >> 1) - 1) & 1,
+                               abort_flag, p.timeout_ns, 2))
+        break;
+      const bool has_k = j < ntiles, has_v = j >= 1;
+      const uint32_t fb = bar.x_full + 8 * b;
+      mbar_arrive_expect_tx_if(leader, fb, (has_k ? C::KT_TX : 0u) + (has_v ? C::V_TX : 0u));
+      if (has_k) {
+        const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
+        const uint32_t dst = sbase + C::OFF_KT + b * C::KT_STAGE;
+#pragma unroll
+        for (int c = 0; c < C::NB; ++c) {
+          tma_load_3d(leader, dst + c * C::KBLK, &p.tm_k, fb, c * 64, key0, bh);
+          tma_load_3d(leader, dst + c * C::KBLK + BN * 128, &p.tm_tk, fb, c * 64, key0, bh);
+        }
+      }
+      if (has_v) {
+        const int32_t key0 = tile_at(j - 1, t0, n0, t2) * BN;
+        const uint32_t dst = sbase + C::OFF_V + ((j - 1) & 1) * C::V_STAGE;
+#pragma unroll
+        for (int c = 0; c < C::NB; ++c) {
+          tma_load_3d(leader, dst + c * C::VBLK, &p.tm_v, fb, c * 64, key0, bh);
+          tma_load_3d(leader, dst + (C::NB + c) * C::VBLK, &p.tm_tv, fb, c * 64, key0, bh);
+        }
+      }
+      steps_armed = j + 1;
+    }
+    // Drain: every copy this warp issued must land before the CTA exits.
+    drain_wait(bar.q_full, 0, p.timeout_ns);
+    for (int32_t j = (steps_armed > 2 ? steps_armed - 2 : 0); j < steps_armed; ++j)
+      drain_wait(bar.x_full + 8 * (j & 1), (j >> 1) & 1, p.timeout_ns);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(BM, 2 * BN, 0);   // Q [K;tK]^T
-      constexpr uint32_t ID_TS = idesc_bf16_f32(BM, BN, 0);      // tQ K^T
-      constexpr uint32_t ID_OT = idesc_bf16_f32(BM, 2 * D, 1);   // P [V|tV]
-      constexpr uint32_t ID_T = idesc_bf16_f32(BM, D, 1);        // (P o tS) V
-      // Operand descriptors: one base per buffer, then compile-time byte offsets
-      // (added to the start-address field, which cannot carry out of its 14 bits
-      // for shared-memory addresses below 256 KiB).
-      const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
-      const uint64_t dTQ = sdesc_sw128(sbase + C::OFF_TQ, 16, 1024);
-      const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_KT, 16, 1024);
-      // MN-major B: 64-element column blocks C::VBLK apart, 8-key groups 1 KiB apart.
-      const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::VBLK, 1024);
-      const uint32_t tS0 = tmem + C::COL_S0;
-      bool ok = wait_bounded(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
-      // Step j: scores of key tile j, then value products of key tile j-1. One
-      // probe covers K(j) and V(j-1); a second one waits for P(j-1).
-      for (int32_t j = 0; ok && j <= ntiles; ++j) {
-        if (!wait_bounded(bar.x_full + 8 * (j & 1), (j >> 1) & 1, abort_flag, p.timeout_ns, 4)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (j < ntiles) {
-          const uint64_t dK = dK0 + uint64_t(((j & 1) * C::KT_STAGE) >> 4);
-          const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
+    // Warp-uniform loop; the elected lane issues every MMA and commit (so one
+    // thread's commits track all of them).
+    const uint32_t leader = elect_one();
+    constexpr uint32_t ID_S = idesc_bf16_f32(BM, 2 * BN, 0);   // Q [K;tK]^T
+    constexpr uint32_t ID_TS = idesc_bf16_f32(BM, BN, 0);      // tQ K^T
+    constexpr uint32_t ID_OT = idesc_bf16_f32(BM, 2 * D, 1);   // P [V|tV]
+    constexpr uint32_t ID_T = idesc_bf16_f32(BM, D, 1);        // (P o tS) V
+    // Operand descriptors: one base per buffer, then compile-time byte offsets
+    // (added to the start-address field, which cannot carry out of its 14 bits
+    // for shared-memory addresses below 256 KiB).
+    const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
+    const uint64_t dTQ = sdesc_sw128(sbase + C::OFF_TQ, 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_KT, 16, 1024);
+    // MN-major B: 64-element column blocks C::VBLK apart, 8-key groups 1 KiB apart.
+    const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::VBLK, 1024);
+    const uint32_t tS0 = tmem + C::COL_S0;
+    bool ok = warp_wait(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
+    // Step j: scores of key tile j, then value products of key tile j-1. One
+    // probe covers K(j) and V(j-1); a second one waits for P(j-1).
+    for (int32_t j = 0; ok && j <= ntiles; ++j) {
+      if (!(ok = warp_wait(bar.x_full + 8 * (j & 1), (j >> 1) & 1, abort_flag, p.timeout_ns, 4)))
+        break;
+      if (j < ntiles) {
+        const uint64_t dK = dK0 + uint64_t(((j & 1) * C::KT_STAGE) >> 4);
+        const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
-            const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
-            const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
-            mma_ss(dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
-            mma_ss(dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
-          }
-          tc_commit(bar.s_full + 8 * (j & 1));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
+          const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
+          const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
+          mma_ss(leader, dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
+          mma_ss(leader, dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
         }
-        if (j >= 1) {
-          const int32_t i = j - 1;
-          if (!wait_bounded(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t dV = dV0 + uint64_t(((i & 1) * C::V_STAGE) >> 4);
-          const uint32_t aP = tS0 + (i & 1) * C::BUF_COLS;
-          const uint32_t first = i > 0 ? 1u : 0u;
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
-            const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
-            mma_ts(tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
-            mma_ts(tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
-          }
-          tc_commit(bar.o_done + 8 * (i & 1));
-        }
+        tc_commit(leader, bar.s_full + 8 * (j & 1));
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      tc_commit(bar.drain);
-      drain_wait(bar.drain, 0, p.timeout_ns);
+      if (j >= 1) {
+        const int32_t i = j - 1;
+        if (!(ok = warp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
+          break;
+        tc_fence_after();
+        const uint64_t dV = dV0 + uint64_t(((i & 1) * C::V_STAGE) >> 4);
+        const uint32_t aP = tS0 + (i & 1) * C::BUF_COLS;
+        const uint32_t first = i > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
+          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
+          mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
+          mma_ts(leader, tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
+        }
+        tc_commit(leader, bar.o_done + 8 * (i & 1));
+      }
     }
+    // Drain: all MMAs issued by the elected lane complete before TMEM is freed.
+    tc_commit(leader, bar.drain);
+    drain_wait(bar.drain, 0, p.timeout_ns);
   } else {
     // ------------------------------------------------- softmax + epilogue
     const int g = (warp - 2) >> 2;            // key half of each tile owned by this warpgroup
@@ -375,17 +389,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       float s[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(rs[i]);
-      // Mask only where this half tile is not entirely inside the row's ranges.
-      const bool full = (kh >= a0 && kh + 32 <= b0) || (kh >= a1 && kh + 32 <= b1);
-      uint32_t vis = 0xffffffffu;
-      if (!full) {
-        vis = 0;
+      // Keys of this half tile the row may see; mask only where some are hidden.
+      // Hidden keys get s = -inf (so p = 0) and a zero score tangent (select, so
+      // a non-finite tangent of a hidden key cannot leak in as 0 * inf).
+      const uint32_t vis = range_bits(a0 - kh, b0 - kh) | range_bits(a1 - kh, b1 - kh);
+      if (vis != 0xffffffffu) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int32_t key = kh + i;
-          const bool v = (key >= a0 && key < b0) || (key >= a1 && key < b1);
-          vis |= uint32_t(v) << i;
+          const bool v = (vis >> i) & 1u;
           s[i] = v ? s[i] : -INFINITY;
+          rt[i] = v ? rt[i] : 0u;
         }
       }
       float mx[8];
@@ -439,33 +452,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this half's first 16 score columns.
       float ls[4] = {0.f, 0.f, 0.f, 0.f}, rsum[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[16], tk[16];
-      if (full) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-          const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
-          const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
-          ls[i & 3] += pa + pb;
-          rsum[i & 3] += qa + qb;
-          pk[i] = pack_bf16(pa, pb);
-          tk[i] = pack_bf16(qa, qb);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-          // invisible keys carry no tangent: select rather than multiply, so a
-          // non-finite score tangent of a masked key cannot leak in as 0 * inf
-          const float ta = ((vis >> (2 * i)) & 1u) ? __uint_as_float(rt[2 * i]) * scale : 0.f;
-          const float tb = ((vis >> (2 * i + 1)) & 1u) ? __uint_as_float(rt[2 * i + 1]) * scale : 0.f;
-          const float qa = pa * ta, qb = pb * tb;
-          ls[i & 3] += pa + pb;
-          rsum[i & 3] += qa + qb;
-          pk[i] = pack_bf16(pa, pb);
-          tk[i] = pack_bf16(qa, qb);
-        }
+      for (int i = 0; i < 16; ++i) {
+        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+        const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
+        const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
+        ls[i & 3] += pa + pb;
+        rsum[i & 3] += qa + qb;
+        pk[i] = pack_bf16(pa, pb);
+        tk[i] = pack_bf16(qa, qb);
       }
       tmem_st16(cS, pk);
       tmem_st16(cT, tk);
