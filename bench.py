@@ -34,6 +34,22 @@ DENSE_BF16_SPEC_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
+# DRAM bytes per launch of the tensor-core kernel on the TF frame-wise workload,
+# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by a
+# hash of the kernel sources it was taken on: a changed kernel reports null.
+KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "kernels.h"]
+MEASURED_TRAFFIC = {}  # {(workload, sources_sha256): bytes per launch}
+
+
+def kernel_sources_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "masked_attention_jvp_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -262,7 +278,9 @@ def bench_gpu(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": args.steps,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": MEASURED_TRAFFIC.get((w.name, kernel_sources_hash())),
+                     "kernel_sources_sha256": kernel_sources_hash(),
                      "peak_source": f"{src} bf16 burst (cuBLAS)", "kernel": "fwd_jvp_sm100_kernel<128>"},
     }
     if world == 1 and not args.no_cpu_baseline:

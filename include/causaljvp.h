@@ -99,6 +99,18 @@ caj_status caj_last_device_status(void *stream);
  * caj_last_device_status returned CAJ_ERR_DEVICE_TIMEOUT. */
 uint32_t caj_last_device_error_code(void);
 
+/* Sets the limit, in milliseconds, on every bounded wait inside the kernels of
+ * later calls on this process (default 2000, or the CAJ_WAIT_TIMEOUT_MS
+ * environment variable). ms <= 0 restores the default. Returns CAJ_OK. */
+caj_status caj_set_wait_timeout_ms(double ms);
+
+/* Test hook for the bounded-wait path: mode 1 makes later tensor-core launches
+ * skip the query-tile copies, so the MMA warp's first wait runs out, the kernel
+ * records CAJ_ERR_DEVICE_TIMEOUT (site 3) and every role exits cleanly. Nothing
+ * faults or hangs; outputs of such a call are undefined. mode 0 (default)
+ * restores normal operation. Returns CAJ_OK, or CAJ_ERR_INVALID_ARG. */
+caj_status caj_debug_set_fault(int32_t mode);
+
 /* Human-readable name of a status. Never NULL. */
 const char *caj_status_string(caj_status s);
 

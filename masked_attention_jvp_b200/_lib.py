@@ -15,7 +15,8 @@ CAJ_DTYPE_F32, CAJ_DTYPE_BF16 = 0, 1
 EXPORTED = [
     "caj_attn_fwd_jvp", "caj_last_device_status", "caj_last_device_error_code",
     "caj_status_string", "caj_last_cuda_error", "caj_validate_mask", "caj_visible_pairs",
-    "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version",
+    "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
+    "caj_debug_set_fault",
 ]
 
 
@@ -68,6 +69,10 @@ def lib() -> ctypes.CDLL:
         L.caj_row_key_ranges.restype = ctypes.c_int
         L.caj_qtile_key_tiles.argtypes = [ctypes.POINTER(MaskDescC), i32, i32, i32, ctypes.POINTER(i32)]
         L.caj_qtile_key_tiles.restype = i32
+        L.caj_set_wait_timeout_ms.argtypes = [ctypes.c_double]
+        L.caj_set_wait_timeout_ms.restype = ctypes.c_int
+        L.caj_debug_set_fault.argtypes = [ctypes.c_int32]
+        L.caj_debug_set_fault.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

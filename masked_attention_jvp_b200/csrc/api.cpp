@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -102,7 +103,12 @@ caj_status check_device() {
   return state[dev] == 1 ? CAJ_OK : CAJ_ERR_UNSUPPORTED;
 }
 
+std::atomic<uint64_t> g_timeout_override_ns{0};
+std::atomic<int32_t> g_fault_mode{0};
+
 uint64_t wait_timeout_ns() {
+  const uint64_t o = g_timeout_override_ns.load();
+  if (o) return o;
   static uint64_t ns = [] {
     const char *s = std::getenv("CAJ_WAIT_TIMEOUT_MS");
     double ms = s ? std::atof(s) : 0.0;
@@ -128,6 +134,17 @@ const char *caj_status_string(caj_status s) {
 }
 
 const char *caj_last_cuda_error(void) { return g_cuda_msg; }
+
+caj_status caj_set_wait_timeout_ms(double ms) {
+  g_timeout_override_ns.store(ms > 0.0 ? uint64_t(ms * 1e6) : 0);
+  return CAJ_OK;
+}
+
+caj_status caj_debug_set_fault(int32_t mode) {
+  if (mode != 0 && mode != 1) return CAJ_ERR_INVALID_ARG;
+  g_fault_mode.store(mode);
+  return CAJ_OK;
+}
 
 int32_t caj_version(void) { return 100; }
 
@@ -217,6 +234,7 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   p.scale = scale;
   p.scale_log2e = scale * 1.4426950408889634f;
   p.timeout_ns = wait_timeout_ns();
+  p.fault_mode = g_fault_mode.load();
   // Launch order: query tiles by decreasing number of key tiles (ties: later first).
   std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
   for (int32_t t = 0; t < n_qtiles; ++t) {

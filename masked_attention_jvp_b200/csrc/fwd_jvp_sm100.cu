@@ -59,6 +59,10 @@ constexpr int BN = kBlockN;  // keys per tile
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale once the max grew by 2^8
+// How many k-steps before the end of the score (S) / value (V) MMA batch the MMA
+// warp probes the barrier the next batch needs (0: after the batch).
+constexpr int kProbeLeadS = 0;
+constexpr int kProbeLeadV = 0;
 
 template <int D>
 struct Cfg {
@@ -249,10 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&p.tm_v);
     }
     const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
-    mbar_arrive_expect_tx_if(leader, bar.q_full, C::Q_TX);
-    for (int c = 0; c < C::NB; ++c) {
-      tma_load_3d(leader, sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
-      tma_load_3d(leader, stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
+    const bool load_q = p.fault_mode != 1;  // test hook: leave q_full unarmed
+    if (load_q) {
+      mbar_arrive_expect_tx_if(leader, bar.q_full, C::Q_TX);
+      for (int c = 0; c < C::NB; ++c) {
+        tma_load_3d(leader, sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
+        tma_load_3d(leader, stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
+      }
     }
     // Step j loads K|tK of key tile j (j < ntiles) into K stage j%2 and V|tV
     // of key tile j-1 (j >= 1) into V stage (j-1)%2, completing on x_full[j%2].
@@ -290,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       steps_armed = j + 1;
     }
     // Drain: every copy this warp issued must land before the CTA exits.
-    drain_wait(bar.q_full, 0, p.timeout_ns);
+    if (load_q) drain_wait(bar.q_full, 0, p.timeout_ns);
     for (int32_t j = (steps_armed > 2 ? steps_armed - 2 : 0); j < steps_armed; ++j)
       drain_wait(bar.x_full + 8 * (j & 1), (j >> 1) & 1, p.timeout_ns);
   } else if (warp == 1) {
@@ -313,26 +320,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS0 = tmem + C::COL_S0;
     bool ok = warp_wait(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
     // Step j: scores of key tile j, then value products of key tile j-1. One
-    // probe covers K(j) and V(j-1); a second one waits for P(j-1).
+    // probe covers K(j) and V(j-1), a second one P(j-1). A probe issued while
+    // earlier MMAs are still queued overlaps their execution, so each probe is
+    // placed kProbeLead k-steps before the end of the batch that precedes its use.
+    if (ok) ok = warp_wait(bar.x_full, 0, abort_flag, p.timeout_ns, 4);
     for (int32_t j = 0; ok && j <= ntiles; ++j) {
-      if (!(ok = warp_wait(bar.x_full + 8 * (j & 1), (j >> 1) & 1, abort_flag, p.timeout_ns, 4)))
-        break;
+      const int32_t i = j - 1;  // key tile whose value products this step issues
+      bool have_p = i < 0;
       if (j < ntiles) {
         const uint64_t dK = dK0 + uint64_t(((j & 1) * C::KT_STAGE) >> 4);
         const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
+          if (kk == D / 16 - kProbeLeadS && !have_p) {
+            if (!(ok = warp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
+              break;
+            have_p = true;
+          }
           // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
           const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
           const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
           mma_ss(leader, dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
           mma_ss(leader, dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
         }
+        if (!ok) break;
         tc_commit(leader, bar.s_full + 8 * (j & 1));
       }
-      if (j >= 1) {
-        const int32_t i = j - 1;
-        if (!(ok = warp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
+      const bool next = j + 1 <= ntiles;  // another step follows
+      bool have_x = !next;
+      if (i >= 0) {
+        if (!have_p &&
+            !(ok = warp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
           break;
         tc_fence_after();
         const uint64_t dV = dV0 + uint64_t(((i & 1) * C::V_STAGE) >> 4);
@@ -340,13 +358,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t first = i > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
+          if (kk == BN / 16 - kProbeLeadV && !have_x) {
+            if (!(ok = warp_wait(bar.x_full + 8 * ((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag,
+                                 p.timeout_ns, 4)))
+              break;
+            have_x = true;
+          }
           const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
           const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
           mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
           mma_ts(leader, tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
         }
+        if (!ok) break;
         tc_commit(leader, bar.o_done + 8 * (i & 1));
       }
+      if (!have_x &&
+          !(ok = warp_wait(bar.x_full + 8 * ((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag,
+                           p.timeout_ns, 4)))
+        break;
     }
     // Drain: all MMAs issued by the elected lane complete before TMEM is freed.
     tc_commit(leader, bar.drain);

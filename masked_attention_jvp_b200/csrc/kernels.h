@@ -33,6 +33,7 @@ struct Sm100Params {
   float scale;           // softmax scale
   float scale_log2e;     // scale * log2(e)
   uint64_t timeout_ns;   // bounded-wait limit
+  int32_t fault_mode;    // test hook: 1 = skip the query-tile copies
   uint16_t qtile_order[kMaxQTiles];  // heaviest query tiles first
 };
 

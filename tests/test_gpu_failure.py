@@ -1,0 +1,46 @@
+"""Failure detection on the GPU without a fault: the tensor-core kernel's waits
+are bounded. With the library's test hook the query-tile copies are skipped, so
+the MMA warp's first wait can never complete; the kernel must give up after the
+configured limit, report CAJ_ERR_DEVICE_TIMEOUT through the device error word,
+leave the context usable, and the next normal call must be correct."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import masked_attention_jvp_b200 as caj
+from masked_attention_jvp_b200 import _lib
+from masked_attention_jvp_b200.workloads import MaskDesc, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    L = _lib.lib()
+    w = Workload("fault", 1, 1, 128, MaskDesc(64, 1, 2, 0), torch.bfloat16, seed=5)  # one CTA
+    ins = make_inputs(w, "cuda")
+    caj.device_status()  # clears any earlier error word
+    assert L.caj_set_wait_timeout_ms(100.0) == _lib.CAJ_OK
+    assert L.caj_debug_set_fault(1) == _lib.CAJ_OK
+    try:
+        caj.attn_fwd_jvp(*ins, w.mask)
+        with pytest.raises(caj.CajError) as err:
+            caj.device_status()
+        assert err.value.status == _lib.CAJ_ERR_DEVICE_TIMEOUT
+        assert L.caj_last_device_error_code() & 0xFF00 == 0x100  # a wait site, not another error
+    finally:
+        L.caj_debug_set_fault(0)
+        L.caj_set_wait_timeout_ms(0.0)
+    caj.device_status()  # the error word was cleared by the read above
+    o, to, lse, tlse = caj.attn_fwd_jvp(*ins, w.mask)
+    caj.device_status()
+    ro, rto, rlse, rtlse = oracle.attn_fwd_jvp(*[t.cpu() for t in ins], w.mask)
+    rel = lambda a, b: float(np.linalg.norm(a - b) / np.linalg.norm(b))
+    assert rel(o.float().cpu().numpy(), ro) <= 1e-2
+    assert rel(to.float().cpu().numpy(), rto) <= 1e-2
+
+
+def test_fault_hook_rejects_unknown_modes():
+    L = _lib.lib()
+    assert L.caj_debug_set_fault(7) == _lib.CAJ_ERR_INVALID_ARG
+    assert L.caj_debug_set_fault(0) == _lib.CAJ_OK

@@ -150,3 +150,12 @@ def test_mask_queries_reject_bad_arguments():
 def test_flops_count():
     m = WORKLOADS["wan1.3b_tf_framewise"].mask
     assert caj.flops(1, 12, 128, m) == 12 * 128 * 1_124_323_200 * 12
+
+
+def test_timeout_and_fault_hooks_host_side():
+    L = _lib.lib()
+    assert L.caj_set_wait_timeout_ms(250.0) == _lib.CAJ_OK
+    assert L.caj_set_wait_timeout_ms(0.0) == _lib.CAJ_OK
+    assert L.caj_debug_set_fault(2) == _lib.CAJ_ERR_INVALID_ARG
+    assert L.caj_debug_set_fault(1) == _lib.CAJ_OK
+    assert L.caj_debug_set_fault(0) == _lib.CAJ_OK
