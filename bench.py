@@ -77,6 +77,19 @@ def flops_of(w):
     return flops(w.B, w.H, w.D, w.mask)
 
 
+def ctz_product_flops(w):
+    """Products actually needed when clean tangents vanish (teacher forcing):
+    clean rows 2 products per visible pair (S, PV), noisy rows over clean keys
+    4 (S, tQ K^T, PV, (P o tS) V), noisy rows over their own chunk all 6; each
+    product is 2 D flops per pair."""
+    m = w.mask
+    G, n = m.frames_per_chunk * m.tokens_per_frame, m.n_frames // m.frames_per_chunk
+    clean = G * G * n * (n + 1) // 2
+    noisy_clean = G * G * n * (n - 1) // 2
+    noisy_own = G * G * n
+    return 2 * w.D * (2 * clean + 4 * noisy_clean + 6 * noisy_own) * w.B * w.H
+
+
 # ----------------------------------------------------------------- CPU oracle
 def oracle_rows_flops(w, rows):
     """12 D flops per visible key of each sampled row (same count as the GPU)."""
@@ -218,6 +231,9 @@ def bench_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload]
     host = make_inputs(w, "cpu")
+    if args.clean_tangent_zero:
+        from masked_attention_jvp_b200.workloads import zero_clean_tangents
+        zero_clean_tangents(w, *host[3:])
     ins = [t.to(dev) for t in host]
     o = torch.empty_like(ins[0])
     to = torch.empty_like(ins[0])
@@ -227,7 +243,8 @@ def bench_gpu(args, rank, world, local_rank):
     fl = flops_of(w)
 
     def step():
-        caj.attn_fwd_jvp_out(*ins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream)
+        caj.attn_fwd_jvp_out(*ins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream,
+                             clean_tangent_zero=args.clean_tangent_zero)
 
     for _ in range(args.warmup):
         step()
@@ -283,6 +300,12 @@ def bench_gpu(args, rank, world, local_rank):
                      "kernel_sources_sha256": kernel_sources_hash(),
                      "peak_source": f"{src} bf16 burst (cuBLAS)", "kernel": "fwd_jvp_sm100_kernel<128>"},
     }
+    if args.clean_tangent_zero:
+        line["config"]["clean_tangent_zero"] = True
+        line["products_tflop_per_step"] = round(ctz_product_flops(w) / 1e12, 3)
+        line["roofline"]["achieved"] = round(ctz_product_flops(w) / (kernel_ms / 1e3) / 1e12, 2)
+        line["roofline"]["frac"] = round(line["roofline"]["achieved"] / peak, 4)
+        line["roofline"]["note"] = "achieved counts only the products the kernel must do"
     if world == 1 and not args.no_cpu_baseline:
         tf, dt, nrows, threads, desc = time_oracle(w, host_inputs=host)
         line["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": threads,
@@ -332,6 +355,9 @@ def main():
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--clean-tangent-zero", action="store_true",
+                    help="TF-sCM inputs: zero clean tangents and let the kernel skip vanishing products "
+                         "(value stays dense-equivalent 12*D per visible pair)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

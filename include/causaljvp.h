@@ -65,12 +65,25 @@ typedef struct {
 } caj_mask_desc;
 
 /* Problem shape. dtype is a caj_dtype and applies to q..tv, o and to.
- * scale <= 0 selects 1/sqrt(D). */
+ * scale <= 0 selects 1/sqrt(D). flags is a bitwise OR of caj_flags. */
 typedef struct {
   int32_t B, H, N, D;
   int32_t dtype;
   float scale;
+  int32_t flags;
 } caj_problem;
+
+/*
+ * CAJ_FLAG_CLEAN_TANGENT_ZERO (teacher-forcing layout only): the caller
+ * guarantees that tq, tk and tv are exactly zero on the clean half (token
+ * rows < L). In TF-sCM the clean context has zero tangent and only the noisy
+ * branch follows the teacher velocity (Causal-rCM section 3.1.2, the paragraph
+ * after eq. 17). The kernel then skips every product that vanishes: query tiles
+ * of clean rows compute only the primal (tO = 0, tLSE = 0), and key tiles of
+ * clean tokens skip Q tK^T and P tV. With the guarantee the results equal the
+ * dense definition; without it they do not.
+ */
+typedef enum { CAJ_FLAG_CLEAN_TANGENT_ZERO = 1 } caj_flags;
 
 /*
  * Forward + JVP of block-causal attention (appendix B eq. 42-45, Algorithm 1).

@@ -73,14 +73,19 @@ def device_status(stream: Optional[torch.cuda.Stream] = None):
     _lib.check(_lib.lib().caj_last_device_status(ctypes.c_void_p(s)), "caj_last_device_status")
 
 
-def _problem(q: torch.Tensor, scale: Optional[float]) -> _lib.ProblemC:
+def _problem(q: torch.Tensor, scale: Optional[float], clean_tangent_zero: bool = False) -> _lib.ProblemC:
     B, H, N, D = q.shape
-    return _lib.ProblemC(B, H, N, D, _DTYPES[q.dtype], float(scale) if scale else 0.0)
+    flags = _lib.CAJ_FLAG_CLEAN_TANGENT_ZERO if clean_tangent_zero else 0
+    return _lib.ProblemC(B, H, N, D, _DTYPES[q.dtype], float(scale) if scale else 0.0, flags)
 
 
 def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optional[float] = None,
-                     stream: Optional[torch.cuda.Stream] = None) -> None:
-    """Writes into caller-provided CUDA tensors o, to [B,H,N,D] and lse, tlse [B,H,N] fp32."""
+                     stream: Optional[torch.cuda.Stream] = None, clean_tangent_zero: bool = False) -> None:
+    """Writes into caller-provided CUDA tensors o, to [B,H,N,D] and lse, tlse [B,H,N] fp32.
+
+    clean_tangent_zero: teacher-forcing layout only; the caller guarantees that
+    tq, tk, tv are zero on the clean half, and the kernel skips the products
+    that vanish (clean query tiles compute only the primal)."""
     ins = (q, k, v, tq, tk, tv)
     for t in ins + (o, to, lse, tlse):
         if not t.is_cuda:
@@ -95,7 +100,7 @@ def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optiona
             or tlse.shape != q.shape[:3]:
         raise ValueError("attn_fwd_jvp_out: lse/tlse must be fp32 [B,H,N]")
     s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
-    prob = _problem(q, scale)
+    prob = _problem(q, scale, clean_tangent_zero)
     st = _lib.lib().caj_attn_fwd_jvp(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
                                      ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)),
                                      ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(to.data_ptr()),
@@ -104,8 +109,9 @@ def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optiona
     _lib.check(st)
 
 
-def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None):
-    """Returns (o, to, lse, tlse). See the module docstring."""
+def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
+                 clean_tangent_zero: bool = False):
+    """Returns (o, to, lse, tlse). See the module docstring and attn_fwd_jvp_out."""
     host = not q.is_cuda
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -117,7 +123,7 @@ def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None):
     to = torch.empty_like(q_)
     lse = torch.empty(q_.shape[:3], dtype=torch.float32, device=q_.device)
     tlse = torch.empty_like(lse)
-    attn_fwd_jvp_out(*ins, mask, o, to, lse, tlse, scale=scale)
+    attn_fwd_jvp_out(*ins, mask, o, to, lse, tlse, scale=scale, clean_tangent_zero=clean_tangent_zero)
     if host:
         outs = []
         for t in (o, to, lse, tlse):

@@ -27,7 +27,11 @@ class MaskDescC(ctypes.Structure):
 
 class ProblemC(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
-                ("D", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("D", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("flags", ctypes.c_int32)]
+
+
+CAJ_FLAG_CLEAN_TANGENT_ZERO = 1
 
 
 class CajError(RuntimeError):

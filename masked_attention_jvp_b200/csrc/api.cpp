@@ -190,6 +190,8 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   if (!geom_from_desc(mask, &g) || g.N != prob->N) return CAJ_ERR_INVALID_ARG;
   if (prob->dtype != CAJ_DTYPE_F32 && prob->dtype != CAJ_DTYPE_BF16) return CAJ_ERR_INVALID_ARG;
   if (!(prob->scale >= 0.f) || std::isinf(prob->scale)) return CAJ_ERR_INVALID_ARG;
+  if (prob->flags & ~int32_t(CAJ_FLAG_CLEAN_TANGENT_ZERO)) return CAJ_ERR_INVALID_ARG;
+  if ((prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) && !mask->tf_layout) return CAJ_ERR_INVALID_ARG;
   if (prob->D != 64 && prob->D != 128) return CAJ_ERR_UNSUPPORTED;
   const int64_t BH = int64_t(prob->B) * prob->H;
   if (BH > 65535 || prob->N > (1 << 20)) return CAJ_ERR_UNSUPPORTED;
@@ -235,6 +237,7 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   p.scale_log2e = scale * 1.4426950408889634f;
   p.timeout_ns = wait_timeout_ns();
   p.fault_mode = g_fault_mode.load();
+  p.clean_tangent_zero = (prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) ? 1 : 0;
   // Launch order: query tiles by decreasing number of key tiles (ties: later first).
   std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
   for (int32_t t = 0; t < n_qtiles; ++t) {

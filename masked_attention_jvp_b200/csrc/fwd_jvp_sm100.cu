@@ -191,7 +191,10 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, timeout_ns, site));
 }
 
-template <int D>
+// CTZ: clean-tangent-zero teacher forcing (the caller guarantees tq, tk, tv
+// vanish on rows < L); a separate instantiation so the dense kernel carries no
+// trace of the specialisation.
+template <int D, bool CTZ>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {
   using C = Cfg<D>;
@@ -218,6 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t t0, t1, t2, t3;
   const int32_t ntiles = qtile_key_tiles(p.geom, q0, q1, BN, t0, t1, t2, t3);
   const int32_t n0 = t1 - t0;
+  // Clean-tangent-zero teacher forcing: a tile of clean query rows has no
+  // tangent at all, and a key tile of clean tokens has tK = tV = 0.
+  const bool no_tan = CTZ && q1 <= p.geom.L;
+  auto clean_keys = [&](int32_t key0) { return CTZ && key0 + BN <= p.geom.L; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q_full, 1);
@@ -255,10 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
     const bool load_q = p.fault_mode != 1;  // test hook: leave q_full unarmed
     if (load_q) {
-      mbar_arrive_expect_tx_if(leader, bar.q_full, C::Q_TX);
+      mbar_arrive_expect_tx_if(leader, bar.q_full, no_tan ? C::Q_TX / 2 : C::Q_TX);
       for (int c = 0; c < C::NB; ++c) {
         tma_load_3d(leader, sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
-        tma_load_3d(leader, stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
+        if (!no_tan) tma_load_3d(leader, stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
       }
     }
     // Step j loads K|tK of key tile j (j < ntiles) into K stage j%2 and V|tV
@@ -274,24 +281,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                                abort_flag, p.timeout_ns, 2))
         break;
       const bool has_k = j < ntiles, has_v = j >= 1;
+      const int32_t kkey0 = has_k ? tile_at(j, t0, n0, t2) * BN : 0;
+      const int32_t vkey0 = has_v ? tile_at(j - 1, t0, n0, t2) * BN : 0;
+      const bool k_tan = has_k && !clean_keys(kkey0);  // tK needed
+      const bool v_tan = has_v && !clean_keys(vkey0);  // tV needed
       const uint32_t fb = bar.x_full + 8 * b;
-      mbar_arrive_expect_tx_if(leader, fb, (has_k ? C::KT_TX : 0u) + (has_v ? C::V_TX : 0u));
+      mbar_arrive_expect_tx_if(leader, fb,
+                               (has_k ? (k_tan ? C::KT_TX : C::KT_TX / 2) : 0u) +
+                                   (has_v ? (v_tan ? C::V_TX : C::V_TX / 2) : 0u));
       if (has_k) {
-        const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
         const uint32_t dst = sbase + C::OFF_KT + b * C::KT_STAGE;
 #pragma unroll
         for (int c = 0; c < C::NB; ++c) {
-          tma_load_3d(leader, dst + c * C::KBLK, &p.tm_k, fb, c * 64, key0, bh);
-          tma_load_3d(leader, dst + c * C::KBLK + BN * 128, &p.tm_tk, fb, c * 64, key0, bh);
+          tma_load_3d(leader, dst + c * C::KBLK, &p.tm_k, fb, c * 64, kkey0, bh);
+          if (k_tan)
+            tma_load_3d(leader, dst + c * C::KBLK + BN * 128, &p.tm_tk, fb, c * 64, kkey0, bh);
         }
       }
       if (has_v) {
-        const int32_t key0 = tile_at(j - 1, t0, n0, t2) * BN;
         const uint32_t dst = sbase + C::OFF_V + ((j - 1) & 1) * C::V_STAGE;
 #pragma unroll
         for (int c = 0; c < C::NB; ++c) {
-          tma_load_3d(leader, dst + c * C::VBLK, &p.tm_v, fb, c * 64, key0, bh);
-          tma_load_3d(leader, dst + (C::NB + c) * C::VBLK, &p.tm_tv, fb, c * 64, key0, bh);
+          tma_load_3d(leader, dst + c * C::VBLK, &p.tm_v, fb, c * 64, vkey0, bh);
+          if (v_tan)
+            tma_load_3d(leader, dst + (C::NB + c) * C::VBLK, &p.tm_tv, fb, c * 64, vkey0, bh);
         }
       }
       steps_armed = j + 1;
@@ -328,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t i = j - 1;  // key tile whose value products this step issues
       bool have_p = i < 0;
       if (j < ntiles) {
+        const int s_mode = no_tan ? 2 : (clean_keys(tile_at(j, t0, n0, t2) * BN) ? 1 : 0);
         const uint64_t dK = dK0 + uint64_t(((j & 1) * C::KT_STAGE) >> 4);
         const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
 #pragma unroll
@@ -340,8 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
           const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
           const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
-          mma_ss(leader, dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
-          mma_ss(leader, dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
+          if (s_mode == 0) {         // [S | Q tK^T] = Q [K;tK]^T, then tS += tQ K^T
+            mma_ss(leader, dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
+            mma_ss(leader, dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
+          } else if (s_mode == 1) {  // clean keys (tK = 0): S = Q K^T, tS = tQ K^T
+            mma_ss(leader, dS, dQ + qo, dK + ko, ID_TS, kk > 0 ? 1u : 0u);
+            mma_ss(leader, dS + BN, dTQ + qo, dK + ko, ID_TS, kk > 0 ? 1u : 0u);
+          } else {                   // no tangent in this query tile: S = Q K^T only
+            mma_ss(leader, dS, dQ + qo, dK + ko, ID_TS, kk > 0 ? 1u : 0u);
+          }
         }
         if (!ok) break;
         tc_commit(leader, bar.s_full + 8 * (j & 1));
@@ -356,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dV = dV0 + uint64_t(((i & 1) * C::V_STAGE) >> 4);
         const uint32_t aP = tS0 + (i & 1) * C::BUF_COLS;
         const uint32_t first = i > 0 ? 1u : 0u;
+        const int v_mode = no_tan ? 2 : (clean_keys(tile_at(i, t0, n0, t2) * BN) ? 1 : 0);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           if (kk == BN / 16 - kProbeLeadV && !have_x) {
@@ -366,8 +388,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
           const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
-          mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
-          mma_ts(leader, tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
+          if (v_mode == 0) {         // [O | T] += P [V | tV], then T += (P o tS) V
+            mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
+            mma_ts(leader, tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
+          } else if (v_mode == 1) {  // clean keys (tV = 0): O += P V, T += (P o tS) V
+            mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_T, kk > 0 ? 1u : first);
+            mma_ts(leader, tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, kk > 0 ? 1u : first);
+          } else {                   // no tangent: O += P V only
+            mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_T, kk > 0 ? 1u : first);
+          }
         }
         if (!ok) break;
         tc_commit(leader, bar.o_done + 8 * (i & 1));
@@ -414,7 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t cS = lane_addr + C::COL_S0 + b * C::BUF_COLS + 32 * g;
       const uint32_t cT = cS + BN;
       uint32_t rs[32], rt[32];
-      tmem_ld32x2(cS, cT, rs, rt);
+      if (no_tan) {  // no score tangent was computed for this query tile
+        tmem_ld32(cS, rs);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rt[i] = 0u;
+      } else {
+        tmem_ld32x2(cS, cT, rs, rt);
+      }
       float s[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(rs[i]);
@@ -481,19 +516,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this half's first 16 score columns.
       float ls[4] = {0.f, 0.f, 0.f, 0.f}, rsum[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[16], tk[16];
+      if (no_tan) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-        const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
-        const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
-        ls[i & 3] += pa + pb;
-        rsum[i & 3] += qa + qb;
-        pk[i] = pack_bf16(pa, pb);
-        tk[i] = pack_bf16(qa, qb);
+        for (int i = 0; i < 16; ++i) {
+          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+          ls[i & 3] += pa + pb;
+          pk[i] = pack_bf16(pa, pb);
+        }
+        tmem_st16(cS, pk);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+          const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
+          const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
+          ls[i & 3] += pa + pb;
+          rsum[i & 3] += qa + qb;
+          pk[i] = pack_bf16(pa, pb);
+          tk[i] = pack_bf16(qa, qb);
+        }
+        tmem_st16(cS, pk);
+        tmem_st16(cT, tk);
       }
-      tmem_st16(cS, pk);
-      tmem_st16(cT, tk);
       l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       r_run += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
       tmem_wait_st();
@@ -530,7 +576,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
           uint32_t ro[32], rt[32];
-          tmem_ld32x2(lane_addr + C::COL_O + c, lane_addr + C::COL_T + c, ro, rt);
+          if (no_tan) {  // T was never written: tO = 0
+            tmem_ld32(lane_addr + C::COL_O + c, ro);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rt[i] = 0u;
+          } else {
+            tmem_ld32x2(lane_addr + C::COL_O + c, lane_addr + C::COL_T + c, ro, rt);
+          }
           uint32_t po[16], pt[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -566,26 +618,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool CTZ>
 cudaError_t launch_impl(const Sm100Params &p, cudaStream_t stream) {
   using C = Cfg<D>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D, CTZ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
-  fwd_jvp_sm100_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  fwd_jvp_sm100_kernel<D, CTZ><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream) {
-  if (D == 128) return launch_impl<128>(p, stream);
-  if (D == 64) return launch_impl<64>(p, stream);
+  const bool ctz = p.clean_tangent_zero != 0;
+  if (D == 128) return ctz ? launch_impl<128, true>(p, stream) : launch_impl<128, false>(p, stream);
+  if (D == 64) return ctz ? launch_impl<64, true>(p, stream) : launch_impl<64, false>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -34,6 +34,7 @@ struct Sm100Params {
   float scale_log2e;     // scale * log2(e)
   uint64_t timeout_ns;   // bounded-wait limit
   int32_t fault_mode;    // test hook: 1 = skip the query-tile copies
+  int32_t clean_tangent_zero;  // tq, tk, tv vanish on rows < L (teacher-forcing layout)
   uint16_t qtile_order[kMaxQTiles];  // heaviest query tiles first
 };
 

@@ -117,6 +117,17 @@ def make_inputs(w: Workload, device="cpu"):
     return tuple(out)
 
 
+def zero_clean_tangents(w: Workload, tq, tk, tv):
+    """Teacher-forcing sCM inputs: the clean context (rows < L) has zero tangent.
+    Zeroes those rows of tq, tk, tv in place and returns them."""
+    if not w.mask.tf_layout:
+        raise ValueError("clean tangents exist only in the teacher-forcing layout")
+    L = w.mask.n_frames * w.mask.tokens_per_frame
+    for t in (tq, tk, tv):
+        t[:, :, :L] = 0
+    return tq, tk, tv
+
+
 def sample_rows(w: Workload, rows_per_head: int, seed_offset: int = 0):
     """Seeded query rows to check per (b, h): `rows_per_head` rows drawn without
     replacement from [0, N) by a generator seeded from (seed, b, h). Returns an

@@ -192,3 +192,55 @@ def test_rejects_mismatched_inputs_without_launch():
     with pytest.raises(ValueError):
         caj.attn_fwd_jvp(*ins, w.mask)
     caj.device_status()
+
+
+# -------------------------------------- clean-tangent-zero teacher forcing (TF-sCM)
+CTZ = [(MaskDesc(37, 1, 7, 1), 1, 2, 128), (MaskDesc(16, 3, 6, 1), 2, 1, 64),
+       (MaskDesc(200, 2, 4, 1), 1, 1, 128), (MaskDesc(64, 1, 4, 1), 1, 2, 128),
+       (MaskDesc(5, 1, 3, 1), 1, 3, 128)]
+
+
+@pytest.mark.parametrize("case", range(len(CTZ)))
+def test_clean_tangent_zero_matches_dense_definition(case):
+    """With zero clean tangents the skipping kernel equals the oracle's dense
+    definition (and the dense kernel, up to rounding)."""
+    from masked_attention_jvp_b200.workloads import zero_clean_tangents
+    mask, B, H, D = CTZ[case]
+    w = Workload(f"ctz{case}", B, H, D, mask, torch.bfloat16, seed=300 + case, std_tangent=0.5)
+    q, k, v, tq, tk, tv = make_inputs(w, "cuda")
+    zero_clean_tangents(w, tq, tk, tv)
+    outs = caj.attn_fwd_jvp(q, k, v, tq, tk, tv, w.mask, clean_tangent_zero=True)
+    torch.cuda.synchronize()
+    caj.device_status()
+    ref = oracle.attn_fwd_jvp_rows(*[t.cpu() for t in (q, k, v, tq, tk, tv)], w.mask)
+    rows = torch.arange(w.B * w.H * w.N)
+    check_rows(gather(outs, rows, w.D), ref, w.dtype, w.name)
+    L = mask.n_frames * mask.tokens_per_frame
+    o, to, lse, tlse = outs
+    assert torch.all(to[:, :, :L] == 0) and torch.all(tlse[:, :, :L] == 0)
+    dense = caj.attn_fwd_jvp(q, k, v, tq, tk, tv, w.mask)
+    assert torch.allclose(outs[0].float(), dense[0].float(), atol=1e-2, rtol=0)
+    assert torch.allclose(outs[1].float(), dense[1].float(), atol=1e-2, rtol=0)
+
+
+@pytest.mark.parametrize("name", ["wan1.3b_tf_framewise", "wan1.3b_tf_chunkwise"])
+def test_clean_tangent_zero_full_size_sampled(name):
+    from masked_attention_jvp_b200.workloads import zero_clean_tangents
+    w = WORKLOADS[name]
+    q, k, v, tq, tk, tv = make_inputs(w, "cuda")
+    zero_clean_tangents(w, tq, tk, tv)
+    outs = caj.attn_fwd_jvp(q, k, v, tq, tk, tv, w.mask, clean_tangent_zero=True)
+    torch.cuda.synchronize()
+    caj.device_status()
+    rows = torch.unique(torch.cat([sample_rows(w, 256), boundary_rows(w)]))
+    host = [t.cpu() for t in (q, k, v, tq, tk, tv)]
+    del q, k, v, tq, tk, tv
+    ref = oracle.attn_fwd_jvp_rows(*host, w.mask, rows=rows)
+    check_rows(gather(outs, rows, w.D), ref, w.dtype, name)
+
+
+def test_clean_tangent_zero_needs_teacher_forcing_layout():
+    w = Workload("ctzbad", 1, 1, 64, MaskDesc(16, 1, 4, 0), torch.bfloat16, seed=1)
+    ins = make_inputs(w, "cuda")
+    with pytest.raises(caj.CajError):
+        caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=True)

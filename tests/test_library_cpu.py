@@ -100,7 +100,7 @@ def test_schedule_at_full_size_covers_every_row(name):
 
 
 def _call(q=0x10000, o=0x20000, lse=0x30000, prob=None, mask=None):
-    prob = prob or _lib.ProblemC(1, 2, 64, 64, _lib.CAJ_DTYPE_BF16, 0.0)
+    prob = prob or _lib.ProblemC(1, 2, 64, 64, _lib.CAJ_DTYPE_BF16, 0.0, 0)
     mask = mask or _lib.MaskDescC(16, 1, 4, 0)
     vp = ctypes.c_void_p
     return _lib.lib().caj_attn_fwd_jvp(vp(q), vp(q), vp(q), vp(q), vp(q), vp(q),
@@ -127,6 +127,9 @@ def test_argument_validation_launches_nothing():
     assert _call(prob=P(1, 2, 128, 64, bf, 0.0), mask=M(16, 1, 4, 1)) != INV  # TF: N = 2L
     assert _call(prob=P(1, 2, 64, 96, bf, 0.0)) == UNS         # head dim not built
     assert _call(prob=P(700, 100, 64, 64, bf, 0.0)) == UNS     # too many heads
+    assert _call(prob=P(1, 2, 64, 64, bf, 0.0, 1)) == INV      # clean-tangent flag needs TF layout
+    assert _call(prob=P(1, 2, 64, 64, bf, 0.0, 4)) == INV      # unknown flag bit
+    assert _call(prob=P(1, 2, 128, 64, bf, 0.0, 1), mask=M(16, 1, 4, 1)) != INV
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
