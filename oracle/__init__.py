@@ -45,6 +45,9 @@ def _load():
                                                             i64, i64, i64, i32, vp, i64,
                                                             vp, vp, vp, vp, i32]
         lib.oracle_attn_fwd_jvp_rows.restype = i32
+        lib.oracle_qk_norm_rope_jvp.argtypes = [vp] * 6 + [i32, vp, vp, vp, vp, i64, i64, i64, i64,
+                                                           dbl, i32] + [vp] * 6
+        lib.oracle_qk_norm_rope_jvp.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
         _lib = lib
@@ -130,3 +133,26 @@ def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale=None, nthreads=0):
     o, to, lse, tlse = attn_fwd_jvp_rows(q, k, v, tq, tk, tv, mask, scale, None, nthreads)
     return (o.reshape(B, H, N, D), to.reshape(B, H, N, D),
             lse.reshape(B, H, N), tlse.reshape(B, H, N))
+
+
+def qk_norm_rope_jvp(xq, xk, xv, txq, txk, txv, gq, gk, cos, sin, H, eps=1e-6, per_head=False):
+    """fp64 layer prologue: RMSNorm (+ JVP) and rotary embedding of q and k,
+    layout change of all six tensors from [B, N, H*D] to [B, H, N, D].
+    Returns numpy arrays (q, k, v, tq, tk, tv), each [B, H, N, D] float64."""
+    ts = [_as_host(t) for t in (xq, xk, xv, txq, txk, txv)]
+    dtypes = {d for _, d in ts}
+    if len(dtypes) != 1:
+        raise TypeError("oracle: all six inputs must share one dtype")
+    dtype = dtypes.pop()
+    B, N, C = xq.shape
+    D = C // H
+    g = [np.ascontiguousarray(torch.as_tensor(x, dtype=torch.float64).cpu().numpy()) for x in (gq, gk)]
+    tab = [np.ascontiguousarray(torch.as_tensor(x, dtype=torch.float64).cpu().numpy()) for x in (cos, sin)]
+    outs = [np.zeros((B, H, N, D), np.float64) for _ in range(6)]
+    rc = _load().oracle_qk_norm_rope_jvp(*[t.data_ptr() for t, _ in ts], dtype,
+                                         g[0].ctypes.data, g[1].ctypes.data, tab[0].ctypes.data,
+                                         tab[1].ctypes.data, B, N, H, D, float(eps), int(bool(per_head)),
+                                         *[o.ctypes.data for o in outs])
+    if rc != 0:
+        raise ValueError("oracle: rejected arguments")
+    return tuple(outs)

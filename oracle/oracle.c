@@ -192,3 +192,77 @@ int oracle_max_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * Layer prologue in primal-tangent form (Causal-rCM section 3.2.2, "JVP FSDP2":
+ * every layer takes and returns a (primal, tangent) pair). For query and key:
+ *   y  = g * x / r,            r = sqrt(mean_C(x^2) + eps)            (RMSNorm)
+ *   ty = g * (tx / r - x * mean_C(x * tx) / r^3)                      (its JVP)
+ * followed by the rotary embedding of interleaved pairs (2i, 2i+1) of each head,
+ *   (a, b) -> (a cos t - b sin t, a sin t + b cos t),  t = theta[n][i],
+ * which is linear and so rotates the tangent the same way. Values and their
+ * tangents are only re-laid out: [B, N, H*D] -> [B, H, N, D].
+ * The normalisation runs over the whole token (C = H*D, per_head = 0) or over
+ * each head (C = D, per_head = 1).
+ *   x*, t*  : [B, N, H*D] in `dtype` (F64 / F32 / BF16 codes as above)
+ *   gq, gk  : [H*D] double;  cosv, sinv : [N, D/2] double
+ *   outputs : [B, H, N, D] double each (q, k, v, tq, tk, tv)
+ */
+int oracle_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv, const void *txq,
+                            const void *txk, const void *txv, int dtype, const double *gq,
+                            const double *gk, const double *cosv, const double *sinv, int64_t B,
+                            int64_t N, int64_t H, int64_t D, double eps, int per_head, double *q,
+                            double *k, double *v, double *tq, double *tk, double *tv) {
+  if (B <= 0 || N <= 0 || H <= 0 || D <= 0 || (D % 2) || eps < 0) return -1;
+  const int64_t C = H * D;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t n = 0; n < N; ++n) {
+      const int64_t in_row = (b * N + n) * C;
+      for (int which = 0; which < 3; ++which) {
+        const void *x = which == 0 ? xq : which == 1 ? xk : xv;
+        const void *tx = which == 0 ? txq : which == 1 ? txk : txv;
+        double *y = which == 0 ? q : which == 1 ? k : v;
+        double *ty = which == 0 ? tq : which == 1 ? tk : tv;
+        const double *g = which == 0 ? gq : gk;
+        for (int64_t h = 0; h < H; ++h) {
+          /* normalisation statistics over the token or over this head */
+          double r = 1.0, m_xtx = 0.0;
+          if (which < 2) {
+            int64_t lo = per_head ? h * D : 0, len = per_head ? D : C;
+            double ss = 0.0, sxt = 0.0;
+            for (int64_t c = lo; c < lo + len; ++c) {
+              double xc = load_elem(x, dtype, in_row + c);
+              ss += xc * xc;
+              sxt += xc * load_elem(tx, dtype, in_row + c);
+            }
+            r = sqrt(ss / (double)len + eps);
+            m_xtx = sxt / (double)len;
+          }
+          const int64_t out_row = ((b * H + h) * N + n) * D;
+          for (int64_t d = 0; d < D; d += 2) {
+            double a = load_elem(x, dtype, in_row + h * D + d);
+            double bb = load_elem(x, dtype, in_row + h * D + d + 1);
+            double ta = load_elem(tx, dtype, in_row + h * D + d);
+            double tb = load_elem(tx, dtype, in_row + h * D + d + 1);
+            if (which < 2) {
+              double ga = g[h * D + d], gb = g[h * D + d + 1];
+              double na = ga * a / r, nb = gb * bb / r;
+              double tna = ga * (ta / r - a * m_xtx / (r * r * r));
+              double tnb = gb * (tb / r - bb * m_xtx / (r * r * r));
+              double cs = cosv[n * (D / 2) + d / 2], sn = sinv[n * (D / 2) + d / 2];
+              a = na * cs - nb * sn;
+              bb = na * sn + nb * cs;
+              ta = tna * cs - tnb * sn;
+              tb = tna * sn + tnb * cs;
+            }
+            y[out_row + d] = a;
+            y[out_row + d + 1] = bb;
+            ty[out_row + d] = ta;
+            ty[out_row + d + 1] = tb;
+          }
+        }
+      }
+    }
+  return 0;
+}
