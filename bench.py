@@ -199,6 +199,41 @@ def whole_job_tflops(flops_per_rank: int, world: int, steps: int, slowest_ms: fl
     return world * flops_per_rank * steps / (slowest_ms / 1e3) / 1e12
 
 
+# ------------------------------------------------------------------ prologue
+def bench_prologue(w, dev, steps, peaks):
+    """The attention block's prologue in primal-tangent form (QK-RMSNorm + JVP,
+    rotary embedding, re-layout of all six tensors) on the workload's shape:
+    HBM-bound, reported against the measured copy bandwidth."""
+    import masked_attention_jvp_b200 as caj
+    B, N, H, D = w.B, w.N, w.H, w.D
+    C = H * D
+    g = torch.Generator(device=dev).manual_seed(w.seed)
+    xs = [torch.randn(B, N, C, device=dev, generator=g).to(torch.bfloat16) for _ in range(6)]
+    gq = torch.ones(C, device=dev)
+    gk = torch.ones(C, device=dev)
+    inv = 10000.0 ** (-torch.arange(0, D, 2, device=dev, dtype=torch.float32) / D)
+    ang = torch.arange(N, device=dev, dtype=torch.float32)[:, None] * inv[None, :]
+    cos, sin = torch.cos(ang).contiguous(), torch.sin(ang).contiguous()
+    out = [torch.empty(B, H, N, D, dtype=torch.bfloat16, device=dev) for _ in range(6)]
+    for _ in range(3):
+        caj.qk_norm_rope_jvp(*xs, gq, gk, cos, sin, H, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        caj.qk_norm_rope_jvp(*xs, gq, gk, cos, sin, H, out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    algo = 12 * B * N * C * 2 + 2 * N * (D // 2) * 4 + 2 * C * 4
+    gbs = algo / (ms / 1e3) / 1e9
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return {"kernel": "qk_norm_rope_jvp_kernel<%d>" % D, "shape": [B, N, H, D], "ms": round(ms, 4),
+            "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(gbs / peak, 4), "algorithmic_bytes": algo, "traffic": None,
+            "note": "inputs 6 x [B,N,H*D] + outputs 6 x [B,H,N,D] bf16 > L2"}
+
+
 # ------------------------------------------------------------------ GPU arm
 def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
     """Same metric through the public API from pinned host buffers: every step
@@ -300,6 +335,9 @@ def bench_gpu(args, rank, world, local_rank):
                      "kernel_sources_sha256": kernel_sources_hash(),
                      "peak_source": f"{src} bf16 burst (cuBLAS)", "kernel": "fwd_jvp_sm100_kernel<128>"},
     }
+    if not args.no_prologue:
+        line["prologue"] = bench_prologue(w, dev, args.steps, peaks)
+        line["gpu_launches_prologue"] = args.steps
     if args.clean_tangent_zero:
         line["config"]["clean_tangent_zero"] = True
         line["products_tflop_per_step"] = round(ctz_product_flops(w) / 1e12, 3)
@@ -355,6 +393,7 @@ def main():
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-prologue", action="store_true", help="skip the prologue kernel's measurement")
     ap.add_argument("--clean-tangent-zero", action="store_true",
                     help="TF-sCM inputs: zero clean tangents and let the kernel skip vanishing products "
                          "(value stays dense-equivalent 12*D per visible pair)")

@@ -103,6 +103,38 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v,
                             void *o, void *to, float *lse, float *tlse,
                             void *stream);
 
+/*
+ * Attention-block prologue in primal-tangent form. Causal-rCM implements the
+ * JVP layer by layer, each layer taking and returning a (primal, tangent) pair
+ * (section 3.2.2, "JVP FSDP2"). For q and k:
+ *   y  = g * x / r, r = sqrt(mean(x^2) + eps)                    (RMSNorm)
+ *   ty = g * (tx / r - x * mean(x * tx) / r^3)                    (its JVP)
+ * then the rotary embedding of interleaved pairs (2i, 2i+1) of each head by the
+ * angle whose cosine/sine are rope_cos/rope_sin[n][i] (linear: the tangent is
+ * rotated the same way). v and tv are copied. The mean runs over the whole
+ * token (norm_per_head = 0, width H*D) or over each head (1, width D).
+ *   in : xq, xk, xv, txq, txk, txv   [B, N, H*D] bf16 (the projections' layout)
+ *        gq, gk                      [H*D] fp32 RMSNorm gains, 16-byte aligned
+ *        rope_cos, rope_sin          [N, D/2] fp32, 16-byte aligned
+ *   out: q, k, v, tq, tk, tv         [B, H, N, D] bf16 (caj_attn_fwd_jvp's layout)
+ * Supported: D in {64, 128}; H*D a multiple of 256 and at most 8192; eps >= 0.
+ * Returns CAJ_OK once enqueued, CAJ_ERR_INVALID_ARG / CAJ_ERR_UNSUPPORTED
+ * without launching, or CAJ_ERR_CUDA.
+ */
+typedef struct {
+  int32_t B, N, H, D;
+  float eps;
+  int32_t norm_per_head;
+} caj_prologue_shape;
+
+caj_status caj_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv,
+                                const void *txq, const void *txk, const void *txv,
+                                const float *gq, const float *gk,
+                                const float *rope_cos, const float *rope_sin,
+                                const caj_prologue_shape *shape,
+                                void *q, void *k, void *v, void *tq, void *tk, void *tv,
+                                void *stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error word.
  * Returns CAJ_OK, CAJ_ERR_DEVICE_TIMEOUT (a kernel abandoned a wait; its
  * outputs are undefined) or CAJ_ERR_CUDA. */

@@ -27,7 +27,7 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "MaskDesc", "CajError", "visible_pairs",
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "qk_norm_rope_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -133,3 +133,34 @@ def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
         torch.cuda.current_stream().synchronize()
         return tuple(outs)
     return o, to, lse, tlse
+
+
+def qk_norm_rope_jvp(xq, xk, xv, txq, txk, txv, gq, gk, rope_cos, rope_sin, H: int,
+                     eps: float = 1e-6, per_head: bool = False, out=None):
+    """Attention-block prologue in primal-tangent form (see include/causaljvp.h).
+
+    xq..txv: [B, N, H*D] bf16 CUDA tensors (projection outputs); gq, gk: [H*D]
+    fp32 RMSNorm gains; rope_cos, rope_sin: [N, D/2] fp32. Returns
+    (q, k, v, tq, tk, tv), each [B, H, N, D] bf16, ready for attn_fwd_jvp.
+    """
+    ins = (xq, xk, xv, txq, txk, txv)
+    B, N, C = xq.shape
+    if C % H:
+        raise ValueError("qk_norm_rope_jvp: H must divide the channel count")
+    D = C // H
+    for t in ins:
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16 and t.shape == xq.shape):
+            raise ValueError("qk_norm_rope_jvp: inputs must be contiguous bf16 CUDA tensors of one shape")
+    for t, shape in ((gq, (C,)), (gk, (C,)), (rope_cos, (N, D // 2)), (rope_sin, (N, D // 2))):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.float32 and tuple(t.shape) == shape):
+            raise ValueError("qk_norm_rope_jvp: gains [H*D] and rope tables [N, D/2] must be fp32 CUDA tensors")
+    if out is None:
+        out = [torch.empty((B, H, N, D), dtype=torch.bfloat16, device=xq.device) for _ in range(6)]
+    shape = _lib.PrologueShapeC(B, N, H, D, float(eps), 1 if per_head else 0)
+    s = torch.cuda.current_stream(xq.device).cuda_stream
+    st = _lib.lib().caj_qk_norm_rope_jvp(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
+                                         *[ctypes.c_void_p(t.data_ptr()) for t in (gq, gk, rope_cos, rope_sin)],
+                                         ctypes.byref(shape), *[ctypes.c_void_p(t.data_ptr()) for t in out],
+                                         ctypes.c_void_p(s))
+    _lib.check(st, "caj_qk_norm_rope_jvp")
+    return tuple(out)

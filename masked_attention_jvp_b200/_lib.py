@@ -16,7 +16,7 @@ EXPORTED = [
     "caj_attn_fwd_jvp", "caj_last_device_status", "caj_last_device_error_code",
     "caj_status_string", "caj_last_cuda_error", "caj_validate_mask", "caj_visible_pairs",
     "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
-    "caj_debug_set_fault",
+    "caj_debug_set_fault", "caj_qk_norm_rope_jvp",
 ]
 
 
@@ -32,6 +32,11 @@ class ProblemC(ctypes.Structure):
 
 
 CAJ_FLAG_CLEAN_TANGENT_ZERO = 1
+
+
+class PrologueShapeC(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("eps", ctypes.c_float), ("norm_per_head", ctypes.c_int32)]
 
 
 class CajError(RuntimeError):
@@ -77,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.caj_set_wait_timeout_ms.restype = ctypes.c_int
         L.caj_debug_set_fault.argtypes = [ctypes.c_int32]
         L.caj_debug_set_fault.restype = ctypes.c_int
+        L.caj_qk_norm_rope_jvp.argtypes = [vp] * 10 + [ctypes.POINTER(PrologueShapeC)] + [vp] * 7
+        L.caj_qk_norm_rope_jvp.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

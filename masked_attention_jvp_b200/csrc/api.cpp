@@ -254,6 +254,35 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
 }
 
+caj_status caj_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv, const void *txq,
+                                const void *txk, const void *txv, const float *gq, const float *gk,
+                                const float *rope_cos, const float *rope_sin,
+                                const caj_prologue_shape *shape, void *q, void *k, void *v, void *tq,
+                                void *tk, void *tv, void *stream) {
+  if (!shape) return CAJ_ERR_INVALID_ARG;
+  const void *ptrs16[] = {xq, xk, xv, txq, txk, txv, gq, gk, rope_cos, rope_sin, q, k, v, tq, tk, tv};
+  for (const void *p : ptrs16)
+    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
+  if (shape->B <= 0 || shape->N <= 0 || shape->H <= 0 || shape->D <= 0) return CAJ_ERR_INVALID_ARG;
+  if (!(shape->eps >= 0.f) || std::isinf(shape->eps)) return CAJ_ERR_INVALID_ARG;
+  if (shape->norm_per_head != 0 && shape->norm_per_head != 1) return CAJ_ERR_INVALID_ARG;
+  if (shape->D != 64 && shape->D != 128) return CAJ_ERR_UNSUPPORTED;
+  const int64_t C = int64_t(shape->H) * shape->D;
+  if (C % 256 != 0 || C > 8192) return CAJ_ERR_UNSUPPORTED;
+  if (int64_t(shape->B) * shape->N > (int64_t(1) << 31) - 1) return CAJ_ERR_UNSUPPORTED;
+  caj_status st = check_device();
+  if (st != CAJ_OK) return st;
+  caj::PrologueParams p{};
+  p.xq = xq; p.xk = xk; p.xv = xv; p.txq = txq; p.txk = txk; p.txv = txv;
+  p.gq = gq; p.gk = gk; p.rope_cos = rope_cos; p.rope_sin = rope_sin;
+  p.q = q; p.k = k; p.v = v; p.tq = tq; p.tk = tk; p.tv = tv;
+  p.B = shape->B; p.N = shape->N; p.H = shape->H; p.D = shape->D;
+  p.eps = shape->eps;
+  p.per_head = shape->norm_per_head;
+  cudaError_t e = caj::launch_qk_norm_rope_jvp(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+}
+
 caj_status caj_last_device_status(void *stream) {
   uint32_t code = 0;
   cudaError_t e = caj::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &code);

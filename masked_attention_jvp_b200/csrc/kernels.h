@@ -47,9 +47,20 @@ struct SimtParams {
   float scale;
 };
 
+struct PrologueParams {
+  const void *xq, *xk, *xv, *txq, *txk, *txv;  // [B, N, H*D] bf16
+  const float *gq, *gk;                        // [H*D]
+  const float *rope_cos, *rope_sin;            // [N, D/2]
+  void *q, *k, *v, *tq, *tk, *tv;              // [B, H, N, D] bf16
+  int32_t B, N, H, D;
+  float eps;
+  int32_t per_head;
+};
+
 // Each returns the launch's cudaError_t (cudaSuccess when enqueued).
 cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream);
 cudaError_t launch_fwd_jvp_simt_f32(const SimtParams &p, int D, cudaStream_t stream);
+cudaError_t launch_qk_norm_rope_jvp(const PrologueParams &p, cudaStream_t stream);
 
 // Device error word access (defined next to the kernels that write it).
 cudaError_t read_and_clear_device_error(cudaStream_t stream, uint32_t *out);

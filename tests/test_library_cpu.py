@@ -162,3 +162,22 @@ def test_timeout_and_fault_hooks_host_side():
     assert L.caj_debug_set_fault(2) == _lib.CAJ_ERR_INVALID_ARG
     assert L.caj_debug_set_fault(1) == _lib.CAJ_OK
     assert L.caj_debug_set_fault(0) == _lib.CAJ_OK
+
+
+def test_prologue_validation_launches_nothing():
+    L = _lib.lib()
+    S = _lib.PrologueShapeC
+    vp = ctypes.c_void_p
+
+    def call(shape, ptr=0x10000, g=0x20000):
+        return L.caj_qk_norm_rope_jvp(*[vp(ptr)] * 6, vp(g), vp(g), vp(g), vp(g), ctypes.byref(shape),
+                                      *[vp(ptr)] * 6, vp(0))
+    assert call(S(1, 8, 12, 128, 1e-6, 0), ptr=0) == _lib.CAJ_ERR_INVALID_ARG
+    assert call(S(1, 8, 12, 128, 1e-6, 0), ptr=0x10008) == _lib.CAJ_ERR_INVALID_ARG
+    assert call(S(1, 8, 12, 128, 1e-6, 0), g=0x20004) == _lib.CAJ_ERR_INVALID_ARG
+    assert call(S(1, 8, 12, 128, -1.0, 0)) == _lib.CAJ_ERR_INVALID_ARG
+    assert call(S(1, 8, 12, 128, 1e-6, 2)) == _lib.CAJ_ERR_INVALID_ARG
+    assert call(S(0, 8, 12, 128, 1e-6, 0)) == _lib.CAJ_ERR_INVALID_ARG
+    assert call(S(1, 8, 12, 96, 1e-6, 0)) == _lib.CAJ_ERR_UNSUPPORTED
+    assert call(S(1, 8, 3, 64, 1e-6, 0)) == _lib.CAJ_ERR_UNSUPPORTED     # H*D not a multiple of 256
+    assert call(S(1, 8, 128, 128, 1e-6, 0)) == _lib.CAJ_ERR_UNSUPPORTED  # H*D > 8192
