@@ -38,13 +38,16 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by a
 # hash of the kernel sources it was taken on: a changed kernel reports null.
 KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "kernels.h"]
-MEASURED_TRAFFIC = {}  # {(workload, sources_sha256): bytes per launch}
+PROLOGUE_SOURCES = ["prologue.cu", "kernels.h"]
+# {(workload, sources_sha256): dram bytes read + written per launch}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "499d4026234ca805"): 1431095808 + 390169344}
+PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "82720d493811c669"): 1241424896 + 1149951232}
 
 
-def kernel_sources_hash() -> str:
+def kernel_sources_hash(files=KERNEL_SOURCES) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in files:
         with open(os.path.join(ROOT, "masked_attention_jvp_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -230,7 +233,8 @@ def bench_prologue(w, dev, steps, peaks):
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     return {"kernel": "qk_norm_rope_jvp_kernel<%d>" % D, "shape": [B, N, H, D], "ms": round(ms, 4),
             "bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(gbs / peak, 4), "algorithmic_bytes": algo, "traffic": None,
+            "frac": round(gbs / peak, 4), "algorithmic_bytes": algo,
+            "traffic": PROLOGUE_TRAFFIC.get((w.name, kernel_sources_hash(PROLOGUE_SOURCES))),
             "note": "inputs 6 x [B,N,H*D] + outputs 6 x [B,H,N,D] bf16 > L2"}
 
 
