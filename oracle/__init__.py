@@ -48,6 +48,8 @@ def _load():
         lib.oracle_qk_norm_rope_jvp.argtypes = [vp] * 6 + [i32, vp, vp, vp, vp, i64, i64, i64, i64,
                                                            dbl, i32] + [vp] * 6
         lib.oracle_qk_norm_rope_jvp.restype = i32
+        lib.oracle_attn_bwd.argtypes = [vp] * 4 + [i32, i64, i64, i64, dbl, i64, i64, i64, i32] + [vp] * 4
+        lib.oracle_attn_bwd.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
         _lib = lib
@@ -156,3 +158,25 @@ def qk_norm_rope_jvp(xq, xk, xv, txq, txk, txv, gq, gk, cos, sin, H, eps=1e-6, p
     if rc != 0:
         raise ValueError("oracle: rejected arguments")
     return tuple(outs)
+
+
+def attn_bwd(q, k, v, dout, mask, scale=None):
+    """fp64 backward of the masked attention primal: (dq, dk, dv, delta) as numpy
+    arrays [B, H, N, D] (delta [B, H, N] = rowsum(P * dP) = <dO, O>)."""
+    ts = [_as_host(t) for t in (q, k, v, dout)]
+    dtypes = {d for _, d in ts}
+    if len(dtypes) != 1:
+        raise TypeError("oracle: all four inputs must share one dtype")
+    dtype = dtypes.pop()
+    B, H, N, D = q.shape
+    T, c, F, tf = _mask_tuple(mask)
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(D))
+    dq, dk, dv = (np.zeros((B, H, N, D), np.float64) for _ in range(3))
+    delta = np.zeros((B, H, N), np.float64)
+    rc = _load().oracle_attn_bwd(*[t.data_ptr() for t, _ in ts], dtype, B * H, N, D, float(scale),
+                                 T, c, F, tf, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
+                                 delta.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle: rejected arguments")
+    return dq, dk, dv, delta

@@ -266,3 +266,84 @@ int oracle_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv, cons
     }
   return 0;
 }
+
+/*
+ * Backward of the primal masked attention (the student's gradient step in
+ * TF-sCM; the JVP branch itself is stop-gradient). For one head, with
+ * P_ij = softmax_j(scale <q_i, k_j>) over the visible keys and dO the gradient of
+ * the output O = P V:
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = <dO_i, v_j>
+ *   Delta_i = sum_j P_ij dP_ij            (equals <dO_i, O_i>)
+ *   dS_ij = P_ij (dP_ij - Delta_i)
+ *   dQ_i  = scale sum_j dS_ij k_j
+ *   dK_j  = scale sum_i dS_ij q_i
+ * The oracle recomputes P from q and k (it does not take an LSE), two passes per
+ * row, fp64, and accumulates dK and dV row by row (each thread owns one head).
+ *   q, k, v, dout : [BH, N, D] in `dtype`;  dq, dk, dv : [BH, N, D] double
+ *   delta         : [BH, N] double (Delta_i), may be NULL
+ */
+int oracle_attn_bwd(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                    int64_t BH, int64_t N, int64_t D, double scale, int64_t T, int64_t c,
+                    int64_t F, int tf, double *dq, double *dk, double *dv, double *delta) {
+  if (D <= 0 || N <= 0 || BH <= 0) return -1;
+  if (N != F * T * (tf ? 2 : 1)) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    const int64_t head = bh * N * D;
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+    int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+    if (!p || !dp || !keys) {
+#pragma omp atomic write
+      bad = 1;
+    } else {
+      for (int64_t x = 0; x < N * D; ++x) dq[head + x] = dk[head + x] = dv[head + x] = 0.0;
+      for (int64_t i = 0; i < N; ++i) {
+        int64_t nk = 0;
+        for (int64_t j = 0; j < N; ++j)
+          if (oracle_visible(T, c, F, tf, i, j)) keys[nk++] = j;
+        if (nk == 0) {
+          if (delta) delta[bh * N + i] = 0.0;
+          continue;
+        }
+        double m = -INFINITY;
+        for (int64_t a = 0; a < nk; ++a) {
+          double s = 0.0, t = 0.0;
+          for (int64_t d = 0; d < D; ++d) {
+            s += load_elem(q, dtype, head + i * D + d) * load_elem(k, dtype, head + keys[a] * D + d);
+            t += load_elem(dout, dtype, head + i * D + d) * load_elem(v, dtype, head + keys[a] * D + d);
+          }
+          p[a] = scale * s;
+          dp[a] = t;
+          if (p[a] > m) m = p[a];
+        }
+        double Z = 0.0;
+        for (int64_t a = 0; a < nk; ++a) {
+          p[a] = exp(p[a] - m);
+          Z += p[a];
+        }
+        double dl = 0.0;
+        for (int64_t a = 0; a < nk; ++a) {
+          p[a] /= Z;
+          dl += p[a] * dp[a];
+        }
+        if (delta) delta[bh * N + i] = dl;
+        for (int64_t a = 0; a < nk; ++a) {
+          const int64_t j = keys[a];
+          const double ds = p[a] * (dp[a] - dl);
+          for (int64_t d = 0; d < D; ++d) {
+            dv[head + j * D + d] += p[a] * load_elem(dout, dtype, head + i * D + d);
+            dq[head + i * D + d] += scale * ds * load_elem(k, dtype, head + j * D + d);
+            dk[head + j * D + d] += scale * ds * load_elem(q, dtype, head + i * D + d);
+          }
+        }
+      }
+    }
+    free(p);
+    free(dp);
+    free(keys);
+  }
+  return bad ? -1 : 0;
+}
