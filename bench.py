@@ -238,6 +238,38 @@ def bench_prologue(w, dev, steps, peaks):
             "note": "inputs 6 x [B,N,H*D] + outputs 6 x [B,H,N,D] bf16 > L2"}
 
 
+# ------------------------------------------------------------------ backward
+def bench_backward(w, ins, o, lse, steps, peaks):
+    """Backward of the primal attention (delta pre-pass, dQ kernel, dK/dV kernel)
+    on the same workload. Algorithmic work: the five products of the standard
+    count, 10 D flops per visible pair per head (the kernels recompute S and dP
+    once more, 14 D in total)."""
+    import masked_attention_jvp_b200 as caj
+    q, k, v = ins[:3]
+    g = torch.Generator(device=q.device).manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, device=q.device, generator=g).to(torch.bfloat16)
+    for _ in range(3):
+        caj.attn_bwd(q, k, v, o, dout, lse, w.mask, scale=w.scale)
+    torch.cuda.synchronize()
+    caj.device_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        caj.attn_bwd(q, k, v, o, dout, lse, w.mask, scale=w.scale)
+    e1.record()
+    torch.cuda.synchronize()
+    caj.device_status()
+    ms = e0.elapsed_time(e1) / steps
+    pairs = flops_of(w) // (12 * w.D)
+    alg = 10 * w.D * pairs
+    tf = alg / (ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    return {"kernels": ["bwd_delta_kernel", "bwd_dq_kernel", "bwd_dkdv_kernel"], "ms": round(ms, 4),
+            "bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(tf / peak, 4), "flop_count": "10*D per visible pair (5 products)",
+            "executed_products_tflop": round(14 * w.D * pairs / 1e12, 3)}
+
+
 # ------------------------------------------------------------------ GPU arm
 def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
     """Same metric through the public API from pinned host buffers: every step
@@ -339,6 +371,9 @@ def bench_gpu(args, rank, world, local_rank):
                      "kernel_sources_sha256": kernel_sources_hash(),
                      "peak_source": f"{src} bf16 burst (cuBLAS)", "kernel": "fwd_jvp_sm100_kernel<128>"},
     }
+    if not args.no_backward and not args.clean_tangent_zero:
+        line["backward"] = bench_backward(w, ins, o, lse, args.steps, peaks)
+        line["gpu_launches_backward"] = 3 * args.steps
     if not args.no_prologue:
         line["prologue"] = bench_prologue(w, dev, args.steps, peaks)
         line["gpu_launches_prologue"] = args.steps
@@ -398,6 +433,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-prologue", action="store_true", help="skip the prologue kernel's measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward kernels' measurement")
     ap.add_argument("--clean-tangent-zero", action="store_true",
                     help="TF-sCM inputs: zero clean tangents and let the kernel skip vanishing products "
                          "(value stays dense-equivalent 12*D per visible pair)")

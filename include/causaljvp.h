@@ -135,6 +135,24 @@ caj_status caj_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv,
                                 void *q, void *k, void *v, void *tq, void *tk, void *tv,
                                 void *stream);
 
+/*
+ * Backward of the primal block-causal attention: the student's gradient step in
+ * TF-sCM (the JVP branch is stop-gradient and needs none). With
+ * P_ij = exp(scale <q_i, k_j> - LSE_i) on visible pairs and dO the gradient of O:
+ *   dV = P^T dO,  dP = dO V^T,  Delta_i = <dO_i, O_i>,  dS = P o (dP - Delta),
+ *   dQ = scale dS K,  dK = scale dS^T Q.
+ *   in : q, k, v, o, dout      [B,H,N,D] bf16 (o from caj_attn_fwd_jvp)
+ *        lse                   [B,H,N] fp32, natural log (from caj_attn_fwd_jvp)
+ *   out: dq, dk, dv            [B,H,N,D] bf16, fully overwritten
+ *        delta                 [B,H,N] fp32, Delta_i = <dO_i, O_i>
+ * prob->dtype must be CAJ_DTYPE_BF16 and D in {64, 128}; prob->flags must be 0.
+ * Deterministic (no atomics). Returns like caj_attn_fwd_jvp.
+ */
+caj_status caj_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                        const void *dout, const float *lse, const caj_problem *prob,
+                        const caj_mask_desc *mask, void *dq, void *dk, void *dv, float *delta,
+                        void *stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error word.
  * Returns CAJ_OK, CAJ_ERR_DEVICE_TIMEOUT (a kernel abandoned a wait; its
  * outputs are undefined) or CAJ_ERR_CUDA. */
@@ -181,6 +199,16 @@ caj_status caj_row_key_ranges(const caj_mask_desc *mask, int32_t row, int32_t r[
  * ascending and disjoint. Returns the number of tiles, or -1 on a bad argument. */
 int32_t caj_qtile_key_tiles(const caj_mask_desc *mask, int32_t q0, int32_t q1,
                             int32_t block_n, int32_t t[4]);
+
+/* Queries that may attend to key `key` (the transposed mask), as up to two
+ * half-open intervals [r[0], r[1]) and [r[2], r[3]). CAJ_OK or CAJ_ERR_INVALID_ARG. */
+caj_status caj_key_query_ranges(const caj_mask_desc *mask, int32_t key, int32_t r[4]);
+
+/* The query tiles of height `block_q` the backward's key-major kernel visits for
+ * the key tile [k0, k1): up to three ascending disjoint half-open tile ranges
+ * t[0..5]. Returns the number of tiles, or -1 on a bad argument. */
+int32_t caj_ktile_query_tiles(const caj_mask_desc *mask, int32_t k0, int32_t k1,
+                              int32_t block_q, int32_t t[6]);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int32_t caj_version(void);

@@ -27,7 +27,7 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "qk_norm_rope_jvp", "MaskDesc", "CajError", "visible_pairs",
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_bwd", "qk_norm_rope_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -164,3 +164,28 @@ def qk_norm_rope_jvp(xq, xk, xv, txq, txk, txv, gq, gk, rope_cos, rope_sin, H: i
                                          ctypes.c_void_p(s))
     _lib.check(st, "caj_qk_norm_rope_jvp")
     return tuple(out)
+
+
+def attn_bwd(q, k, v, o, dout, lse, mask, scale: Optional[float] = None):
+    """Backward of the primal masked attention (see include/causaljvp.h).
+
+    q, k, v, o, dout: [B, H, N, D] bf16 CUDA tensors (o and lse from
+    attn_fwd_jvp on the same q, k, v). Returns (dq, dk, dv, delta) with
+    delta = rowsum(dout * o) in fp32 [B, H, N]."""
+    ins = (q, k, v, o, dout)
+    for t in ins:
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16 and t.shape == q.shape):
+            raise ValueError("attn_bwd: q, k, v, o, dout must be contiguous bf16 CUDA tensors of one shape")
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.shape == q.shape[:3] and lse.is_contiguous()):
+        raise ValueError("attn_bwd: lse must be a contiguous fp32 CUDA tensor [B, H, N]")
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    delta = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    prob = _problem(q, scale)
+    s = torch.cuda.current_stream(q.device).cuda_stream
+    st = _lib.lib().caj_attn_bwd(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
+                                 ctypes.c_void_p(lse.data_ptr()), ctypes.byref(prob),
+                                 ctypes.byref(_lib.mask_c(mask)),
+                                 *[ctypes.c_void_p(t.data_ptr()) for t in (dq, dk, dv, delta)],
+                                 ctypes.c_void_p(s))
+    _lib.check(st, "caj_attn_bwd")
+    return dq, dk, dv, delta

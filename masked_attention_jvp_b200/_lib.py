@@ -16,7 +16,8 @@ EXPORTED = [
     "caj_attn_fwd_jvp", "caj_last_device_status", "caj_last_device_error_code",
     "caj_status_string", "caj_last_cuda_error", "caj_validate_mask", "caj_visible_pairs",
     "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
-    "caj_debug_set_fault", "caj_qk_norm_rope_jvp",
+    "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
+    "caj_attn_bwd",
 ]
 
 
@@ -84,6 +85,12 @@ def lib() -> ctypes.CDLL:
         L.caj_debug_set_fault.restype = ctypes.c_int
         L.caj_qk_norm_rope_jvp.argtypes = [vp] * 10 + [ctypes.POINTER(PrologueShapeC)] + [vp] * 7
         L.caj_qk_norm_rope_jvp.restype = ctypes.c_int
+        L.caj_key_query_ranges.argtypes = [ctypes.POINTER(MaskDescC), i32, ctypes.POINTER(i32)]
+        L.caj_key_query_ranges.restype = ctypes.c_int
+        L.caj_ktile_query_tiles.argtypes = [ctypes.POINTER(MaskDescC), i32, i32, i32, ctypes.POINTER(i32)]
+        L.caj_ktile_query_tiles.restype = i32
+        L.caj_attn_bwd.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC)] + [vp] * 5
+        L.caj_attn_bwd.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

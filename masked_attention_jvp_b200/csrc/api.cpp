@@ -175,6 +175,23 @@ int32_t caj_qtile_key_tiles(const caj_mask_desc *mask, int32_t q0, int32_t q1, i
   return caj::qtile_key_tiles(g, q0, q1, block_n, t[0], t[1], t[2], t[3]);
 }
 
+caj_status caj_key_query_ranges(const caj_mask_desc *mask, int32_t key, int32_t r[4]) {
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g) || !r || key < 0 || key >= g.N) return CAJ_ERR_INVALID_ARG;
+  caj::key_query_ranges(g, key, r[0], r[1], r[2], r[3]);
+  return CAJ_OK;
+}
+
+int32_t caj_ktile_query_tiles(const caj_mask_desc *mask, int32_t k0, int32_t k1, int32_t block_q,
+                              int32_t t[6]) {
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g) || !t || block_q <= 0 || k0 < 0 || k1 <= k0 || k1 > g.N) return -1;
+  int32_t tt[6];
+  const int32_t n = caj::ktile_query_tiles(g, k0, k1, block_q, tt);
+  for (int i = 0; i < 6; ++i) t[i] = tt[i];
+  return n;
+}
+
 caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const void *tq,
                             const void *tk, const void *tv, const caj_problem *prob,
                             const caj_mask_desc *mask, void *o, void *to, float *lse, float *tlse,
@@ -283,10 +300,78 @@ caj_status caj_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv, 
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
 }
 
+caj_status caj_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                        const void *dout, const float *lse, const caj_problem *prob,
+                        const caj_mask_desc *mask, void *dq, void *dk, void *dv, float *delta,
+                        void *stream) {
+  if (!prob || !mask) return CAJ_ERR_INVALID_ARG;
+  const void *ins[] = {q, k, v, o, dout, dq, dk, dv};
+  for (const void *p : ins)
+    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
+  if (!lse || !delta || !aligned4(lse) || !aligned4(delta)) return CAJ_ERR_INVALID_ARG;
+  if (prob->B <= 0 || prob->H <= 0 || prob->N <= 0 || prob->D <= 0) return CAJ_ERR_INVALID_ARG;
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g) || g.N != prob->N) return CAJ_ERR_INVALID_ARG;
+  if (prob->dtype != CAJ_DTYPE_F32 && prob->dtype != CAJ_DTYPE_BF16) return CAJ_ERR_INVALID_ARG;
+  if (!(prob->scale >= 0.f) || std::isinf(prob->scale)) return CAJ_ERR_INVALID_ARG;
+  if (prob->flags != 0) return CAJ_ERR_INVALID_ARG;
+  if (prob->dtype != CAJ_DTYPE_BF16) return CAJ_ERR_UNSUPPORTED;
+  if (prob->D != 64 && prob->D != 128) return CAJ_ERR_UNSUPPORTED;
+  const int64_t BH = int64_t(prob->B) * prob->H;
+  if (BH > 65535 || prob->N > (1 << 20)) return CAJ_ERR_UNSUPPORTED;
+  const int32_t ntile = (prob->N + caj::kBlockM - 1) / caj::kBlockM;
+  if (ntile > caj::kMaxQTiles) return CAJ_ERR_UNSUPPORTED;
+  caj_status st = check_device();
+  if (st != CAJ_OK) return st;
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+  std::unique_ptr<caj::BwdParams> hp(new caj::BwdParams());
+  caj::BwdParams &p = *hp;
+  const int N = prob->N, D = prob->D;
+  const bool okm = encode_map(enc, &p.tm_q_r, q, int(BH), N, D, 128) &&
+                   encode_map(enc, &p.tm_do_r, dout, int(BH), N, D, 128) &&
+                   encode_map(enc, &p.tm_k_s, k, int(BH), N, D, 64) &&
+                   encode_map(enc, &p.tm_v_s, v, int(BH), N, D, 64) &&
+                   encode_map(enc, &p.tm_k_r, k, int(BH), N, D, 128) &&
+                   encode_map(enc, &p.tm_v_r, v, int(BH), N, D, 128) &&
+                   encode_map(enc, &p.tm_q_s, q, int(BH), N, D, 64) &&
+                   encode_map(enc, &p.tm_do_s, dout, int(BH), N, D, 64);
+  if (!okm) return cuda_fail(cudaErrorInvalidValue);
+  p.o = o; p.dout = dout; p.lse = lse; p.delta = delta; p.dq = dq; p.dk = dk; p.dv = dv;
+  p.geom = g;
+  p.BH = int32_t(BH);
+  p.n_row_tiles = ntile;
+  p.scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt(float(D));
+  p.timeout_ns = wait_timeout_ns();
+  // Launch orders: query tiles by decreasing key-tile count, key tiles by
+  // decreasing query-tile count (ties: later first).
+  std::vector<std::pair<int32_t, int32_t>> cq(ntile), ck(ntile);
+  for (int32_t t = 0; t < ntile; ++t) {
+    int32_t r[6];
+    const int32_t a = t * caj::kBlockM, b = std::min(a + caj::kBlockM, N);
+    cq[t] = {caj::qtile_key_tiles(g, a, b, caj::kBlockN, r[0], r[1], r[2], r[3]), t};
+    ck[t] = {caj::ktile_query_tiles(g, a, b, caj::kBlockN, r), t};
+  }
+  auto heavier = [](const auto &x, const auto &y) {
+    return x.first != y.first ? x.first > y.first : x.second > y.second;
+  };
+  std::sort(cq.begin(), cq.end(), heavier);
+  std::sort(ck.begin(), ck.end(), heavier);
+  for (int32_t i = 0; i < ntile; ++i) {
+    p.row_order[i] = uint16_t(cq[i].second);
+    p.col_order[i] = uint16_t(ck[i].second);
+  }
+  cudaError_t e = caj::launch_attn_bwd_sm100(p, D, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+}
+
 caj_status caj_last_device_status(void *stream) {
-  uint32_t code = 0;
+  uint32_t code = 0, bcode = 0;
   cudaError_t e = caj::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &code);
   if (e != cudaSuccess) return cuda_fail(e);
+  e = caj::read_and_clear_bwd_error(&bcode);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!code) code = bcode;
   if (code != 0) {
     g_last_device_code = code;
     return CAJ_ERR_DEVICE_TIMEOUT;

@@ -57,10 +57,29 @@ struct PrologueParams {
   int32_t per_head;
 };
 
+struct BwdParams {
+  // dq kernel: resident Q, dO (128-row boxes), streamed K, V (64-row boxes);
+  // dkdv kernel: resident K, V (128-row boxes), streamed Q, dO (64-row boxes)
+  CUtensorMap tm_q_r, tm_do_r, tm_k_s, tm_v_s, tm_k_r, tm_v_r, tm_q_s, tm_do_s;
+  const void *o, *dout;   // [B*H, N, D] bf16 (for Delta)
+  const float *lse;       // [B*H, N] natural log, from the forward
+  float *delta;           // [B*H, N] Delta = <dO, O> (written by the pre-pass)
+  void *dq, *dk, *dv;     // [B*H, N, D] bf16
+  MaskGeom geom;
+  int32_t BH;
+  int32_t n_row_tiles;    // ceil(N / 128), for both query and key tiles
+  float scale;
+  uint64_t timeout_ns;
+  uint16_t row_order[kMaxQTiles];  // query tiles, heaviest first (dq kernel)
+  uint16_t col_order[kMaxQTiles];  // key tiles, heaviest first (dkdv kernel)
+};
+
 // Each returns the launch's cudaError_t (cudaSuccess when enqueued).
 cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream);
 cudaError_t launch_fwd_jvp_simt_f32(const SimtParams &p, int D, cudaStream_t stream);
 cudaError_t launch_qk_norm_rope_jvp(const PrologueParams &p, cudaStream_t stream);
+cudaError_t launch_attn_bwd_sm100(const BwdParams &p, int D, cudaStream_t stream);
+cudaError_t read_and_clear_bwd_error(uint32_t *out);
 
 // Device error word access (defined next to the kernels that write it).
 cudaError_t read_and_clear_device_error(cudaStream_t stream, uint32_t *out);

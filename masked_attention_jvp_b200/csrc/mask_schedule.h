@@ -83,6 +83,84 @@ CAJ_HD int32_t qtile_key_tiles(const MaskGeom &m, int32_t q0, int32_t q1, int32_
   return (t1 - t0) + (t3 - t2);
 }
 
+// Queries that may attend to key `k` (the transposed mask), as up to two
+// intervals [a0, b0) U [a1, b1):
+//   plain layout, key in chunk j:     [j G, N)
+//   clean key in chunk j (TF layout): clean queries [j G, L) and noisy queries
+//                                     of later chunks [L + (j+1) G, 2L)
+//   noisy key in chunk j (TF layout): the noisy queries of chunk j
+CAJ_HD void key_query_ranges(const MaskGeom &m, int32_t k, int32_t &a0, int32_t &b0, int32_t &a1,
+                             int32_t &b1) {
+  if (!m.tf) {
+    a0 = (k / m.G) * m.G;
+    b0 = m.N;
+    a1 = b1 = 0;
+  } else if (k < m.L) {
+    const int32_t j = k / m.G;
+    a0 = j * m.G;
+    b0 = m.L;
+    a1 = m.L + (j + 1) * m.G;
+    b1 = 2 * m.L;
+    if (a1 >= b1) a1 = b1 = 0;
+  } else {
+    const int32_t j = (k - m.L) / m.G;
+    a0 = m.L + j * m.G;
+    b0 = a0 + m.G;
+    a1 = b1 = 0;
+  }
+}
+
+// Query tiles of height bq that some key of [k0, k1) is visible to, as up to
+// three ascending disjoint tile ranges t[0..5] ([t0,t1) U [t2,t3) U [t4,t5)).
+// Returns the number of tiles.
+CAJ_HD int32_t ktile_query_tiles(const MaskGeom &m, int32_t k0, int32_t k1, int32_t bq,
+                                 int32_t (&t)[6]) {
+  // Query intervals of the union: the first key of each part has the widest.
+  int32_t lo[3], hi[3], n = 0;
+  if (!m.tf) {
+    lo[n] = (k0 / m.G) * m.G;
+    hi[n++] = m.N;
+  } else {
+    if (k0 < m.L) {  // clean keys: the earliest chunk sees the most queries
+      const int32_t j = k0 / m.G;
+      lo[n] = j * m.G;
+      hi[n++] = m.L;
+      if (m.L + (j + 1) * m.G < 2 * m.L) {
+        lo[n] = m.L + (j + 1) * m.G;
+        hi[n++] = 2 * m.L;
+      }
+    }
+    if (k1 > m.L) {  // noisy keys: queries of the noisy chunks they span
+      const int32_t first = k0 > m.L ? k0 : m.L;
+      const int32_t e0 = (first - m.L) / m.G, e1 = (k1 - 1 - m.L) / m.G;
+      lo[n] = m.L + e0 * m.G;
+      hi[n++] = m.L + (e1 + 1) * m.G;
+    }
+  }
+  // sort the (at most three) intervals by start, then merge in tile units
+  for (int32_t a = 0; a < n; ++a)
+    for (int32_t b = a + 1; b < n; ++b)
+      if (lo[b] < lo[a]) {
+        int32_t x = lo[a]; lo[a] = lo[b]; lo[b] = x;
+        x = hi[a]; hi[a] = hi[b]; hi[b] = x;
+      }
+  int32_t r = 0;
+  for (int32_t a = 0; a < n; ++a) {
+    const int32_t s = lo[a] / bq, e = (hi[a] + bq - 1) / bq;
+    if (r > 0 && s <= t[2 * r - 1]) {
+      if (e > t[2 * r - 1]) t[2 * r - 1] = e;
+    } else {
+      t[2 * r] = s;
+      t[2 * r + 1] = e;
+      ++r;
+    }
+  }
+  int32_t total = 0;
+  for (int32_t a = 0; a < r; ++a) total += t[2 * a + 1] - t[2 * a];
+  for (int32_t a = r; a < 3; ++a) t[2 * a] = t[2 * a + 1] = (r ? t[2 * r - 1] : 0);
+  return total;
+}
+
 // Visible (query, key) pairs of one head: n chunks of G tokens; chunk j of the
 // plain layout sees j+1 chunks (G^2 n(n+1)/2 in all); the teacher-forcing
 // layout adds the same count again for the noisy copy.

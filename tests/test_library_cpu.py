@@ -181,3 +181,33 @@ def test_prologue_validation_launches_nothing():
     assert call(S(1, 8, 12, 96, 1e-6, 0)) == _lib.CAJ_ERR_UNSUPPORTED
     assert call(S(1, 8, 3, 64, 1e-6, 0)) == _lib.CAJ_ERR_UNSUPPORTED     # H*D not a multiple of 256
     assert call(S(1, 8, 128, 128, 1e-6, 0)) == _lib.CAJ_ERR_UNSUPPORTED  # H*D > 8192
+
+
+@pytest.mark.parametrize("mask", MASKS)
+def test_key_ranges_match_oracle_visibility(mask):
+    """The transposed mask: queries that see each key, against brute force."""
+    L = _lib.lib()
+    N = mask.seq_len
+    r = (ctypes.c_int32 * 4)()
+    for j in range(N):
+        assert L.caj_key_query_ranges(ctypes.byref(_lib.mask_c(mask)), j, r) == _lib.CAJ_OK
+        got = set(range(r[0], r[1])) | set(range(r[2], r[3]))
+        want = {i for i in range(N) if oracle.visible(mask, i, j)}
+        assert got == want, (mask, j)
+
+
+@pytest.mark.parametrize("mask", MASKS)
+@pytest.mark.parametrize("bk,bq", [(128, 64), (16, 8), (7, 5), (64, 128)])
+def test_key_tile_schedule_matches_brute_force(mask, bk, bq):
+    """The key-major backward visits exactly the query tiles that see some key of the tile."""
+    L = _lib.lib()
+    N = mask.seq_len
+    t = (ctypes.c_int32 * 6)()
+    for k0 in range(0, N, bk):
+        k1 = min(k0 + bk, N)
+        n = L.caj_ktile_query_tiles(ctypes.byref(_lib.mask_c(mask)), k0, k1, bq, t)
+        tiles = list(range(t[0], t[1])) + list(range(t[2], t[3])) + list(range(t[4], t[5]))
+        assert t[0] <= t[1] <= t[2] <= t[3] <= t[4] <= t[5]
+        assert n == len(tiles)
+        want = sorted({i // bq for j in range(k0, k1) for i in range(N) if oracle.visible(mask, i, j)})
+        assert tiles == want, (mask, k0, k1, bk, bq)
