@@ -297,15 +297,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       uint32_t rs[32], rp[32];
       tmem_ld32x2(cS, cS + 64, rs, rp);
       const uint32_t vis = bits_in(a0 - kh, b0 - kh) | bits_in(a1 - kh, b1 - kh);
+      if (vis != 0xffffffffu) {  // hidden keys: p = 0 and no dP (select, NaN-safe)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool v = (vis >> i) & 1u;
+          rs[i] = v ? rs[i] : __float_as_uint(-INFINITY);
+          rp[i] = v ? rp[i] : __float_as_uint(dl);
+        }
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const bool va = (vis >> (2 * i)) & 1u, vb = (vis >> (2 * i + 1)) & 1u;
-        const float pa = va ? ex2(fmaf(__uint_as_float(rs[2 * i]), sl2, -lse2)) : 0.f;
-        const float pb = vb ? ex2(fmaf(__uint_as_float(rs[2 * i + 1]), sl2, -lse2)) : 0.f;
-        const float da = va ? __uint_as_float(rp[2 * i]) - dl : 0.f;
-        const float db = vb ? __uint_as_float(rp[2 * i + 1]) - dl : 0.f;
-        pk[i] = pack_bf16(pa * da, pb * db);
+        const float pa = ex2(fmaf(__uint_as_float(rs[2 * i]), sl2, -lse2));
+        const float pb = ex2(fmaf(__uint_as_float(rs[2 * i + 1]), sl2, -lse2));
+        pk[i] = pack_bf16(pa * (__uint_as_float(rp[2 * i]) - dl), pb * (__uint_as_float(rp[2 * i + 1]) - dl));
       }
       tmem_st16(cS, pk);
       tmem_wait_st();
@@ -481,6 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       uint32_t rs[32], rp[32];
       tmem_ld32x2(cS, cS + 64, rs, rp);
       const uint32_t vis = bits_in(a0 - qh, b0 - qh) | bits_in(a1 - qh, b1 - qh);
+      if (vis != 0xffffffffu) {  // queries that do not see this key: p = 0, no dP
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool v = (vis >> i) & 1u;
+          rs[i] = v ? rs[i] : __float_as_uint(-INFINITY);
+          rp[i] = v ? rp[i] : 0u;
+        }
+      }
       const float4 *st4 = reinterpret_cast<const float4 *>(sgen + C::OFF_ST + s * C::STAGE +
                                                            2 * C::S_BYTES) + 8 * g;
       uint32_t pk[16], dk[16];
@@ -491,11 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int i = 2 * i4 + h, c0 = 2 * i, c1 = 2 * i + 1;
-          const bool va = (vis >> c0) & 1u, vb = (vis >> c1) & 1u;
-          const float pa = va ? ex2(fmaf(__uint_as_float(rs[c0]), sl2, -lv[2 * h])) : 0.f;
-          const float pb = vb ? ex2(fmaf(__uint_as_float(rs[c1]), sl2, -lv[2 * h + 1])) : 0.f;
-          const float da = va ? __uint_as_float(rp[c0]) - dv[2 * h] : 0.f;
-          const float db = vb ? __uint_as_float(rp[c1]) - dv[2 * h + 1] : 0.f;
+          // hidden pairs: s = -inf gives p = 0, so dS = 0 whatever dP - Delta is
+          const float pa = ex2(fmaf(__uint_as_float(rs[c0]), sl2, -lv[2 * h]));
+          const float pb = ex2(fmaf(__uint_as_float(rs[c1]), sl2, -lv[2 * h + 1]));
+          const float da = __uint_as_float(rp[c0]) - dv[2 * h];
+          const float db = __uint_as_float(rp[c1]) - dv[2 * h + 1];
           pk[i] = pack_bf16(pa, pb);
           dk[i] = pack_bf16(pa * da, pb * db);
         }
