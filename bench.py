@@ -37,19 +37,31 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # DRAM bytes per launch of the tensor-core kernel on the TF frame-wise workload,
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by a
 # hash of the kernel sources it was taken on: a changed kernel reports null.
-KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "kernels.h"]
-PROLOGUE_SOURCES = ["prologue.cu", "kernels.h"]
+# each kernel's sources plus the parameter struct it is launched with
+KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct Sm100Params"]
+PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
+BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
 # {(workload, sources_sha256): dram bytes read + written per launch}
-MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "499d4026234ca805"): 1431095808 + 390169344}
-PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "82720d493811c669"): 1241424896 + 1149951232}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "30f728faff142e26"): 1426396928 + 390678528}
+PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241282560 + 1150534656}
+# summed over the three launches of one backward call (delta, dQ, dK/dV)
+BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "46f5460b56276709"):
+                    402563840 + 5564416 + 815246336 + 184427520 + 816951808 + 384215040}
 
 
 def kernel_sources_hash(files=KERNEL_SOURCES) -> str:
     import hashlib
+    import re
+    csrc = os.path.join(ROOT, "masked_attention_jvp_b200", "csrc")
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "masked_attention_jvp_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        if f.startswith("struct "):
+            text = open(os.path.join(csrc, "kernels.h")).read()
+            m = re.search(r"^%s \{.*?^\};" % re.escape(f), text, re.S | re.M)
+            h.update(m.group(0).encode() if m else f.encode())
+        else:
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -267,6 +279,7 @@ def bench_backward(w, ins, o, lse, steps, peaks):
     return {"kernels": ["bwd_delta_kernel", "bwd_dq_kernel", "bwd_dkdv_kernel"], "ms": round(ms, 4),
             "bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(tf / peak, 4), "flop_count": "10*D per visible pair (5 products)",
+            "traffic": BACKWARD_TRAFFIC.get((w.name, kernel_sources_hash(BACKWARD_SOURCES))),
             "executed_products_tflop": round(14 * w.D * pairs / 1e12, 3)}
 
 
