@@ -328,16 +328,14 @@ caj_status caj_attn_bwd(const void *q, const void *k, const void *v, const void 
   std::unique_ptr<caj::BwdParams> hp(new caj::BwdParams());
   caj::BwdParams &p = *hp;
   const int N = prob->N, D = prob->D;
-  const bool okm = encode_map(enc, &p.tm_q_r, q, int(BH), N, D, 128) &&
-                   encode_map(enc, &p.tm_do_r, dout, int(BH), N, D, 128) &&
-                   encode_map(enc, &p.tm_k_s, k, int(BH), N, D, 64) &&
+  // q, k and dout are also read row by row with 16-byte loads (checked above)
+  const bool okm = encode_map(enc, &p.tm_k_s, k, int(BH), N, D, 64) &&
                    encode_map(enc, &p.tm_v_s, v, int(BH), N, D, 64) &&
-                   encode_map(enc, &p.tm_k_r, k, int(BH), N, D, 128) &&
                    encode_map(enc, &p.tm_v_r, v, int(BH), N, D, 128) &&
                    encode_map(enc, &p.tm_q_s, q, int(BH), N, D, 64) &&
                    encode_map(enc, &p.tm_do_s, dout, int(BH), N, D, 64);
   if (!okm) return cuda_fail(cudaErrorInvalidValue);
-  p.o = o; p.dout = dout; p.lse = lse; p.delta = delta; p.dq = dq; p.dk = dk; p.dv = dv;
+  p.q = q; p.k = k; p.o = o; p.dout = dout; p.lse = lse; p.delta = delta; p.dq = dq; p.dk = dk; p.dv = dv;
   p.geom = g;
   p.BH = int32_t(BH);
   p.n_row_tiles = ntile;

@@ -19,6 +19,11 @@
 // copies, warp 1 the MMAs (elected lane, warp-uniform loop), warps 2-9 form two
 // warpgroups that each take one 32-column half of every 64-column tile. P and
 // dS are written back to TMEM as bf16 over the columns their thread read.
+// The CTA's own 128 rows that serve as the A operand of the score products
+// (Q and dO in dq, K in dkdv) are copied once into TMEM by the softmax warps,
+// so those N = 64 products read only the streamed 64-row tile from shared
+// memory: shared-memory bandwidth, not the tensor core, bounded them when A
+// came from shared memory too.
 // Every mbarrier wait is bounded; on expiry the kernel records an error code,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -41,7 +46,6 @@ constexpr int BM = 128;  // rows owned by a CTA (queries for dq, keys for dkdv)
 constexpr int BN = 64;   // streamed tile width (keys for dq, queries for dkdv)
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
-constexpr int kStages = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __noinline__ void bwd_raise(volatile int *abort_flag, uint32_t code) {
@@ -96,22 +100,24 @@ __device__ __forceinline__ int32_t nth_tile(int32_t j, const int32_t (&t)[6]) {
   return t[4] + (j - n0 - n1);
 }
 
-template <int D>
+// NRES: resident 128-row tiles kept in shared memory (0 in dq, V in dkdv).
+template <int D, int NRES>
 struct BCfg {
   static constexpr int NB = D / 64;          // 128-byte column blocks per row
   static constexpr int RBLK = BM * 128;      // one column block of a resident 128-row tile
   static constexpr int SBLK = BN * 128;      // one column block of a streamed 64-row tile
   static constexpr int R_BYTES = NB * RBLK;  // a resident 128 x D tile
   static constexpr int S_BYTES = NB * SBLK;  // a streamed 64 x D tile
+  static constexpr int STAGES = 4;
   // stage: two streamed tiles + 2 x 64 fp32 row statistics (dkdv), padded so
   // every stage starts on a 1 KiB boundary (128-byte swizzle)
   static constexpr int STAGE = 2 * S_BYTES + 1024;
-  static constexpr int OFF_R0 = 0;
-  static constexpr int OFF_R1 = R_BYTES;
-  static constexpr int OFF_ST = 2 * R_BYTES;
-  static constexpr int OFF_BAR = OFF_ST + kStages * STAGE;
-  // barriers: r_full, st_full[3], st_empty[3], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int NBAR = 1 + 2 * kStages + 7;
+  static constexpr int OFF_R = 0;
+  static constexpr int OFF_ST = NRES * R_BYTES;
+  static constexpr int OFF_BAR = OFF_ST + STAGES * STAGE;
+  // barriers: a_ready, r_full, st_full[S], st_empty[S], s_full[2], p_full[2],
+  // o_done[2], drain, dp_free
+  static constexpr int NBAR = 2 + 2 * STAGES + 8;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
@@ -119,31 +125,59 @@ struct BCfg {
 };
 
 struct BBars {
-  uint32_t r_full, st_full, st_empty, s_full, p_full, o_done, drain;
+  uint32_t a_ready, r_full, st_full, st_empty, s_full, p_full, o_done, drain, dp_free;
 };
 
+template <int STAGES>
 __device__ __forceinline__ BBars bbars(uint32_t base) {
   BBars b;
-  b.r_full = base;
-  b.st_full = base + 8;
-  b.st_empty = b.st_full + 8 * kStages;
-  b.s_full = b.st_empty + 8 * kStages;
+  b.a_ready = base;
+  b.r_full = base + 8;
+  b.st_full = base + 16;
+  b.st_empty = b.st_full + 8 * STAGES;
+  b.s_full = b.st_empty + 8 * STAGES;
   b.p_full = b.s_full + 16;
   b.o_done = b.p_full + 16;
   b.drain = b.o_done + 16;
+  b.dp_free = b.drain + 8;
   return b;
+}
+
+// Copies half g of this thread's bf16 row into TMEM as packed pairs: column
+// taddr + i holds elements (2i, 2i+1) of the row, the layout in which the
+// tensor core reads an A operand from TMEM (one 16-element K step per 8
+// columns). Rows past the sequence are zero, as a TMA copy would fill them.
+template <int D>
+__device__ __forceinline__ void row_to_tmem(const uint16_t *row, bool live, uint32_t taddr, int g) {
+  constexpr int W = D / 4;  // 32-bit words in half a row
+  uint32_t w[W];
+  const uint4 *s4 = reinterpret_cast<const uint4 *>(row) + g * (W / 4);
+#pragma unroll
+  for (int v = 0; v < W / 4; ++v) {
+    const uint4 x = live ? __ldg(s4 + v) : make_uint4(0u, 0u, 0u, 0u);
+    w[4 * v] = x.x;
+    w[4 * v + 1] = x.y;
+    w[4 * v + 2] = x.z;
+    w[4 * v + 3] = x.w;
+  }
+  if constexpr (W == 32) {
+    tmem_st32(taddr + g * W, w);
+  } else {
+    tmem_st16(taddr + g * W, w);
+  }
 }
 
 // Shared prologue of both kernels: barriers, TMEM, error checks. Returns false
 // when the CTA must return at once.
-template <int D>
+template <class C>
 __device__ __forceinline__ bool bwd_setup(uint32_t sbase, uint8_t *sgen, const BBars &bar,
                                           int warp) {
-  using C = BCfg<D>;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + C::OFF_MISC + 4);
   if (threadIdx.x == 0) {
+    mbar_init(bar.a_ready, kSoftmaxWarps);
     mbar_init(bar.r_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    mbar_init(bar.dp_free, kSoftmaxWarps);
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar.st_full + 8 * s, 1);
       mbar_init(bar.st_empty + 8 * s, 1);
     }
@@ -169,7 +203,7 @@ __device__ __forceinline__ bool bwd_setup(uint32_t sbase, uint8_t *sgen, const B
 // ============================================================== dQ kernel
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
-  using C = BCfg<D>;
+  using C = BCfg<D, 0>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   if (sbase & 1023u) {
@@ -177,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     return;
   }
   uint8_t *sgen = smem_raw;
-  const BBars bar = bbars(sbase + C::OFF_BAR);
+  const BBars bar = bbars<C::STAGES>(sbase + C::OFF_BAR);
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sgen + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + C::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -189,24 +223,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
   const int32_t ntiles = qtile_key_tiles(p.geom, q0, q1, BN, t[0], t[1], t[2], t[3]);
   t[4] = t[5] = t[3];
 
-  bwd_setup<D>(sbase, sgen, bar, warp);
+  bwd_setup<C>(sbase, sgen, bar, warp);
   const uint32_t tmem = *tmem_slot;
-  // TMEM: dQ accumulator [0, D) | buffer b: S [D + 128b, +64), dP [+64, +128)
-  const uint32_t COL_S0 = D;
+  // TMEM: dQ accumulator [0, D) | Q [D, 3D/2) | dO [3D/2, 2D) (packed bf16, the
+  // A operands of the score products) | buffer b: S [2D + 128b, +64), dP [+64, +128)
+  constexpr uint32_t COL_Q = D, COL_DO = D + D / 2, COL_S0 = 2 * D;
+  static_assert(COL_S0 + 256 <= C::TMEM_COLS, "TMEM overflow");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint32_t leader = elect_one();
-    mbar_arrive_expect_tx_if(leader, bar.r_full, 2 * C::R_BYTES);
-    for (int c = 0; c < C::NB; ++c) {
-      tma_load_3d(leader, sbase + C::OFF_R0 + c * C::RBLK, &p.tm_q_r, bar.r_full, c * 64, q0, bh);
-      tma_load_3d(leader, sbase + C::OFF_R1 + c * C::RBLK, &p.tm_do_r, bar.r_full, c * 64, q0, bh);
-    }
     int32_t armed = 0;
     for (int32_t j = 0; j < ntiles; ++j) {
-      const int s = j % kStages;
-      if (j >= kStages && !bwarp_wait(bar.st_empty + 8 * s, ((j / kStages) - 1) & 1, abort_flag,
-                                      p.timeout_ns, 21))
+      const int s = j % C::STAGES;
+      if (j >= C::STAGES && !bwarp_wait(bar.st_empty + 8 * s, ((j / C::STAGES) - 1) & 1, abort_flag,
+                                        p.timeout_ns, 21))
         break;
       const int32_t key0 = nth_tile(j, t) * BN;
       const uint32_t dst = sbase + C::OFF_ST + s * C::STAGE, fb = bar.st_full + 8 * s;
@@ -218,33 +249,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       }
       armed = j + 1;
     }
-    bdrain(bar.r_full, 0, p.timeout_ns);
-    for (int32_t j = (armed > kStages ? armed - kStages : 0); j < armed; ++j)
-      bdrain(bar.st_full + 8 * (j % kStages), (j / kStages) & 1, p.timeout_ns);
+    for (int32_t j = (armed > C::STAGES ? armed - C::STAGES : 0); j < armed; ++j)
+      bdrain(bar.st_full + 8 * (j % C::STAGES), (j / C::STAGES) & 1, p.timeout_ns);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     const uint32_t leader = elect_one();
     constexpr uint32_t ID_S = idesc_bf16_f32(BM, BN, 0);  // Q K^T, dO V^T
     constexpr uint32_t ID_Q = idesc_bf16_f32(BM, D, 1);   // dS K, K read MN-major
-    const uint64_t dQ = sdesc_sw128(sbase + C::OFF_R0, 16, 1024);
-    const uint64_t dO = sdesc_sw128(sbase + C::OFF_R1, 16, 1024);
     const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_ST, 16, 1024);
     const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_ST + C::S_BYTES, 16, 1024);
     const uint64_t dKmn0 = sdesc_sw128(sbase + C::OFF_ST, C::SBLK, 1024);
-    bool ok = bwarp_wait(bar.r_full, 0, abort_flag, p.timeout_ns, 22);
+    bool ok = bwarp_wait(bar.a_ready, 0, abort_flag, p.timeout_ns, 22);
+    tc_fence_after();
     for (int32_t j = 0; ok && j <= ntiles; ++j) {
       if (j < ntiles) {
-        const int s = j % kStages;
-        if (!(ok = bwarp_wait(bar.st_full + 8 * s, (j / kStages) & 1, abort_flag, p.timeout_ns, 23)))
+        const int s = j % C::STAGES;
+        if (!(ok = bwarp_wait(bar.st_full + 8 * s, (j / C::STAGES) & 1, abort_flag, p.timeout_ns, 23)))
           break;
         const uint64_t so = uint64_t((s * C::STAGE) >> 4);
         const uint32_t cS = tmem + COL_S0 + (j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ro = uint64_t(((kk >> 2) * C::RBLK + (kk & 3) * 32) >> 4);
           const uint64_t st = uint64_t(((kk >> 2) * C::SBLK + (kk & 3) * 32) >> 4);
-          mma_ss(leader, cS, dQ + ro, dK0 + so + st, ID_S, kk > 0 ? 1u : 0u);
-          mma_ss(leader, cS + 64, dO + ro, dV0 + so + st, ID_S, kk > 0 ? 1u : 0u);
+          mma_ts(leader, cS, tmem + COL_Q + 8 * kk, dK0 + so + st, ID_S, kk > 0 ? 1u : 0u);
+          mma_ts(leader, cS + 64, tmem + COL_DO + 8 * kk, dV0 + so + st, ID_S, kk > 0 ? 1u : 0u);
         }
         tc_commit(leader, bar.s_full + 8 * (j & 1));
       }
@@ -253,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
         if (!(ok = bwarp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 24)))
           break;
         tc_fence_after();
-        const int s = i % kStages;
+        const int s = i % C::STAGES;
         const uint64_t so = uint64_t((s * C::STAGE) >> 4);
         const uint32_t aS = tmem + COL_S0 + (i & 1) * 128;
 #pragma unroll
@@ -284,6 +312,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       a0 = 0; b0 = p.geom.N; a1 = b1 = 0;
     }
     const float sl2 = p.scale * kLog2e;
+    {  // this thread's rows of Q and dO become the A operands in TMEM
+      const size_t off = (size_t(bh) * p.geom.N + (live ? q : 0)) * D;
+      row_to_tmem<D>(static_cast<const uint16_t *>(p.q) + off, live, lane_addr + COL_Q, g);
+      row_to_tmem<D>(static_cast<const uint16_t *>(p.dout) + off, live, lane_addr + COL_DO, g);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.a_ready);
+    }
     bool ok = true;
     for (int32_t j = 0; j < ntiles; ++j) {
       const int b = j & 1;
@@ -351,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
 // ============================================================ dK dV kernel
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
-  using C = BCfg<D>;
+  using C = BCfg<D, 1>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   if (sbase & 1023u) {
@@ -359,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     return;
   }
   uint8_t *sgen = smem_raw;
-  const BBars bar = bbars(sbase + C::OFF_BAR);
+  const BBars bar = bbars<C::STAGES>(sbase + C::OFF_BAR);
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sgen + C::OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + C::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -370,24 +407,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
   int32_t t[6];
   const int32_t ntiles = ktile_query_tiles(p.geom, k0, k1, BN, t);
 
-  bwd_setup<D>(sbase, sgen, bar, warp);
+  bwd_setup<C>(sbase, sgen, bar, warp);
   const uint32_t tmem = *tmem_slot;
-  // TMEM: dV [0, D) | dK [D, 2D) | buffer b: S^T [2D + 128b, +64), dP^T [+64, +128)
-  const uint32_t COL_S0 = 2 * D;
+  // TMEM: dV [0, D) | dK [D, 2D) | K [2D, 5D/2) (packed bf16, the A operand of
+  // S^T) | buffer b: S^T [COL_S0 + 64b, +64), then P^T and dS^T packed over it
+  // | dP^T [COL_S0 + 128, +64), one buffer, free once the softmax has read it
+  constexpr uint32_t COL_K = 2 * D, COL_S0 = (5 * D / 2 + 63) / 64 * 64, COL_DP = COL_S0 + 128;
+  static_assert(COL_DP + 64 <= C::TMEM_COLS, "TMEM overflow");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint32_t leader = elect_one();
-    mbar_arrive_expect_tx_if(leader, bar.r_full, 2 * C::R_BYTES);
-    for (int c = 0; c < C::NB; ++c) {
-      tma_load_3d(leader, sbase + C::OFF_R0 + c * C::RBLK, &p.tm_k_r, bar.r_full, c * 64, k0, bh);
-      tma_load_3d(leader, sbase + C::OFF_R1 + c * C::RBLK, &p.tm_v_r, bar.r_full, c * 64, k0, bh);
-    }
+    mbar_arrive_expect_tx_if(leader, bar.r_full, C::R_BYTES);
+    for (int c = 0; c < C::NB; ++c)
+      tma_load_3d(leader, sbase + C::OFF_R + c * C::RBLK, &p.tm_v_r, bar.r_full, c * 64, k0, bh);
     int32_t armed = 0;
     for (int32_t j = 0; j < ntiles; ++j) {
-      const int s = j % kStages;
-      if (j >= kStages && !bwarp_wait(bar.st_empty + 8 * s, ((j / kStages) - 1) & 1, abort_flag,
-                                      p.timeout_ns, 31))
+      const int s = j % C::STAGES;
+      if (j >= C::STAGES && !bwarp_wait(bar.st_empty + 8 * s, ((j / C::STAGES) - 1) & 1, abort_flag,
+                                        p.timeout_ns, 31))
         break;
       const int32_t qb = nth_tile(j, t) * BN;
       const uint32_t dst = sbase + C::OFF_ST + s * C::STAGE, fb = bar.st_full + 8 * s;
@@ -411,33 +449,43 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       armed = j + 1;
     }
     bdrain(bar.r_full, 0, p.timeout_ns);
-    for (int32_t j = (armed > kStages ? armed - kStages : 0); j < armed; ++j)
-      bdrain(bar.st_full + 8 * (j % kStages), (j / kStages) & 1, p.timeout_ns);
+    for (int32_t j = (armed > C::STAGES ? armed - C::STAGES : 0); j < armed; ++j)
+      bdrain(bar.st_full + 8 * (j % C::STAGES), (j / C::STAGES) & 1, p.timeout_ns);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     const uint32_t leader = elect_one();
     constexpr uint32_t ID_S = idesc_bf16_f32(BM, BN, 0);  // K Q^T, V dO^T
     constexpr uint32_t ID_A = idesc_bf16_f32(BM, D, 1);   // P^T dO, dS^T Q (B read MN-major)
-    const uint64_t dK = sdesc_sw128(sbase + C::OFF_R0, 16, 1024);
-    const uint64_t dV = sdesc_sw128(sbase + C::OFF_R1, 16, 1024);
+    const uint64_t dV = sdesc_sw128(sbase + C::OFF_R, 16, 1024);
     const uint64_t dQ0 = sdesc_sw128(sbase + C::OFF_ST, 16, 1024);
     const uint64_t dO0 = sdesc_sw128(sbase + C::OFF_ST + C::S_BYTES, 16, 1024);
     const uint64_t dQmn0 = sdesc_sw128(sbase + C::OFF_ST, C::SBLK, 1024);
     const uint64_t dOmn0 = sdesc_sw128(sbase + C::OFF_ST + C::S_BYTES, C::SBLK, 1024);
-    bool ok = bwarp_wait(bar.r_full, 0, abort_flag, p.timeout_ns, 32);
+    bool ok = bwarp_wait(bar.a_ready, 0, abort_flag, p.timeout_ns, 38) &&
+              bwarp_wait(bar.r_full, 0, abort_flag, p.timeout_ns, 32);
+    tc_fence_after();
     for (int32_t j = 0; ok && j <= ntiles; ++j) {
       if (j < ntiles) {
-        const int s = j % kStages;
-        if (!(ok = bwarp_wait(bar.st_full + 8 * s, (j / kStages) & 1, abort_flag, p.timeout_ns, 33)))
+        const int s = j % C::STAGES;
+        if (!(ok = bwarp_wait(bar.st_full + 8 * s, (j / C::STAGES) & 1, abort_flag, p.timeout_ns, 33)))
           break;
         const uint64_t so = uint64_t((s * C::STAGE) >> 4);
-        const uint32_t cS = tmem + COL_S0 + (j & 1) * 128;
+        const uint32_t cS = tmem + COL_S0 + (j & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t st = uint64_t(((kk >> 2) * C::SBLK + (kk & 3) * 32) >> 4);
+          mma_ts(leader, cS, tmem + COL_K + 8 * kk, dQ0 + so + st, ID_S, kk > 0 ? 1u : 0u);
+        }
+        // dP^T has one buffer: the softmax must have read dP^T(j-1)
+        if (j >= 1) {
+          if (!(ok = bwarp_wait(bar.dp_free, (j - 1) & 1, abort_flag, p.timeout_ns, 39))) break;
+          tc_fence_after();
+        }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ro = uint64_t(((kk >> 2) * C::RBLK + (kk & 3) * 32) >> 4);
           const uint64_t st = uint64_t(((kk >> 2) * C::SBLK + (kk & 3) * 32) >> 4);
-          mma_ss(leader, cS, dK + ro, dQ0 + so + st, ID_S, kk > 0 ? 1u : 0u);
-          mma_ss(leader, cS + 64, dV + ro, dO0 + so + st, ID_S, kk > 0 ? 1u : 0u);
+          mma_ss(leader, tmem + COL_DP, dV + ro, dO0 + so + st, ID_S, kk > 0 ? 1u : 0u);
         }
         tc_commit(leader, bar.s_full + 8 * (j & 1));
       }
@@ -446,16 +494,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         if (!(ok = bwarp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 34)))
           break;
         tc_fence_after();
-        const int s = i % kStages;
+        const int s = i % C::STAGES;
         const uint64_t so = uint64_t((s * C::STAGE) >> 4);
-        const uint32_t aP = tmem + COL_S0 + (i & 1) * 128;
+        const uint32_t aP = tmem + COL_S0 + (i & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;  // packed columns of queries 16kk..
+          // queries 16kk.. : warpgroup kk>>1 packed P^T at +0 and dS^T at +16 of its 32 columns
+          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;
           const uint64_t ko = uint64_t((kk * 16 * 128) >> 4);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
           mma_ts(leader, tmem, aP + pc, dOmn0 + so + ko, ID_A, acc);           // dV += P^T dO
-          mma_ts(leader, tmem + D, aP + 64 + pc, dQmn0 + so + ko, ID_A, acc);  // dK += dS^T Q
+          mma_ts(leader, tmem + D, aP + 16 + pc, dQmn0 + so + ko, ID_A, acc);  // dK += dS^T Q
         }
         tc_commit(leader, bar.o_done + 8 * (i & 1));
         tc_commit(leader, bar.st_empty + 8 * s);
@@ -472,19 +521,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     int32_t a0 = 0, b0 = 0, a1 = 0, b1 = 0;  // queries that see this key (none past N)
     if (live) key_query_ranges(p.geom, key, a0, b0, a1, b1);
     const float sl2 = p.scale * kLog2e;
+    {  // this thread's row of K becomes the A operand of S^T in TMEM
+      const size_t off = (size_t(bh) * p.geom.N + (live ? key : 0)) * D;
+      row_to_tmem<D>(static_cast<const uint16_t *>(p.k) + off, live, lane_addr + COL_K, g);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.a_ready);
+    }
     bool ok = true;
     for (int32_t j = 0; j < ntiles; ++j) {
-      const int b = j & 1, s = j % kStages;
+      const int b = j & 1, s = j % C::STAGES;
       if (!bwarp_wait(bar.s_full + 8 * b, (j >> 1) & 1, abort_flag, p.timeout_ns, 35) ||
-          !bwarp_wait(bar.st_full + 8 * s, (j / kStages) & 1, abort_flag, p.timeout_ns, 36)) {
+          !bwarp_wait(bar.st_full + 8 * s, (j / C::STAGES) & 1, abort_flag, p.timeout_ns, 36)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int32_t qh = nth_tile(j, t) * BN + 32 * g;
-      const uint32_t cS = lane_addr + COL_S0 + b * 128 + 32 * g;
+      const uint32_t cS = lane_addr + COL_S0 + b * 64 + 32 * g;
       uint32_t rs[32], rp[32];
-      tmem_ld32x2(cS, cS + 64, rs, rp);
+      tmem_ld32x2(cS, lane_addr + COL_DP + 32 * g, rs, rp);
+      tc_fence_before();  // dP^T is in registers: its buffer may be overwritten
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.dp_free);
       const uint32_t vis = bits_in(a0 - qh, b0 - qh) | bits_in(a1 - qh, b1 - qh);
       if (vis != 0xffffffffu) {  // queries that do not see this key: p = 0, no dP
 #pragma unroll
@@ -514,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         }
       }
       tmem_st16(cS, pk);
-      tmem_st16(cS + 64, dk);
+      tmem_st16(cS + 16, dk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -590,14 +650,15 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const void *o, const voi
 
 template <int D>
 cudaError_t launch_bwd_impl(const BwdParams &p, cudaStream_t stream) {
-  using C = BCfg<D>;
+  using CQ = BCfg<D, 0>;
+  using CK = BCfg<D, 1>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
+                                         CQ::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES);
+                             CK::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -607,12 +668,12 @@ cudaError_t launch_bwd_impl(const BwdParams &p, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(p.n_row_tiles) * unsigned(p.BH);
-  bwd_dq_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  bwd_dq_kernel<D><<<grid, kThreads, CQ::SMEM_BYTES, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   BwdParams pk = p;  // the key-major kernel takes the key-tile order
   for (int32_t i = 0; i < p.n_row_tiles; ++i) pk.row_order[i] = p.col_order[i];
-  bwd_dkdv_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(pk);
+  bwd_dkdv_kernel<D><<<grid, kThreads, CK::SMEM_BYTES, stream>>>(pk);
   return cudaGetLastError();
 }
 

@@ -58,10 +58,12 @@ struct PrologueParams {
 };
 
 struct BwdParams {
-  // dq kernel: resident Q, dO (128-row boxes), streamed K, V (64-row boxes);
-  // dkdv kernel: resident K, V (128-row boxes), streamed Q, dO (64-row boxes)
-  CUtensorMap tm_q_r, tm_do_r, tm_k_s, tm_v_s, tm_k_r, tm_v_r, tm_q_s, tm_do_s;
-  const void *o, *dout;   // [B*H, N, D] bf16 (for Delta)
+  // dq kernel: streamed K, V (64-row boxes); Q and dO rows are read into TMEM;
+  // dkdv kernel: resident V (128-row box), streamed Q, dO (64-row boxes); K
+  // rows are read into TMEM
+  CUtensorMap tm_k_s, tm_v_s, tm_v_r, tm_q_s, tm_do_s;
+  const void *q, *k;      // [B*H, N, D] bf16
+  const void *o, *dout;   // [B*H, N, D] bf16 (o for Delta only)
   const float *lse;       // [B*H, N] natural log, from the forward
   float *delta;           // [B*H, N] Delta = <dO, O> (written by the pre-pass)
   void *dq, *dk, *dv;     // [B*H, N, D] bf16
