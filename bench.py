@@ -42,11 +42,11 @@ KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struc
 PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
 BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
 # {(workload, sources_sha256): dram bytes read + written per launch}
-MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "30f728faff142e26"): 1426396928 + 390678528}
-PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241282560 + 1150534656}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "eb9dbceb765b4a8c"): 1428671488 + 390379008}
+PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241276160 + 1150380544}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
-BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "46f5460b56276709"):
-                    402563840 + 5564416 + 815246336 + 184427520 + 816951808 + 384215040}
+BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "97e98721674f6154"):
+                    402571008 + 5875712 + 813365248 + 184498432 + 815200768 + 383543296}
 
 
 def kernel_sources_hash(files=KERNEL_SOURCES) -> str:
@@ -313,7 +313,7 @@ def bench_gpu(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = WORKLOADS[args.workload]
+    w = selected_workload(args)
     host = make_inputs(w, "cpu")
     if args.clean_tangent_zero:
         from masked_attention_jvp_b200.workloads import zero_clean_tangents
@@ -409,7 +409,7 @@ def bench_reference(args, rank):
         return None
     import oracle
     from masked_attention_jvp_b200.workloads import sample_rows
-    w = WORKLOADS[args.workload]
+    w = selected_workload(args)
     host = make_inputs(w, "cpu")
     threads = oracle.max_threads()
     per_head = 8
@@ -436,6 +436,14 @@ def bench_reference(args, rank):
     }
 
 
+def selected_workload(args):
+    import dataclasses
+    w = WORKLOADS[args.workload]
+    if args.heads is not None:
+        w = dataclasses.replace(w, name=f"{w.name}_h{args.heads}", H=args.heads)
+    return w
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -447,6 +455,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-prologue", action="store_true", help="skip the prologue kernel's measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward kernels' measurement")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (small cases for ncu section captures)")
     ap.add_argument("--clean-tangent-zero", action="store_true",
                     help="TF-sCM inputs: zero clean tangents and let the kernel skip vanishing products "
                          "(value stays dense-equivalent 12*D per visible pair)")

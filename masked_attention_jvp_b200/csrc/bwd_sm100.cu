@@ -16,14 +16,21 @@
 //              (the transposed block-causal schedule): S^T = K Q^T and
 //              dP^T = V dO^T, then dV += P^T dO and dK += dS^T Q.
 // Both main kernels reuse the forward kernel's organisation: warp 0 issues TMA
-// copies, warp 1 the MMAs (elected lane, warp-uniform loop), warps 2-9 form two
+// copies, warp 1 the MMAs (elected lane, warp-uniform loop). Warps 2-9 form two
 // warpgroups that each take one 32-column half of every 64-column tile. P and
-// dS are written back to TMEM as bf16 over the columns their thread read.
+// dS are written back to TMEM as bf16 over the columns their thread read. (Four
+// warpgroups of 16 columns each, 576 threads, measured 8% slower: the softmax
+// is bound by the exponential unit and by fixed load/store/barrier latencies,
+// which more warps do not shorten, and the extra warps share sub-partitions
+// with the copy and MMA warps.)
 // The CTA's own 128 rows that serve as the A operand of the score products
 // (Q and dO in dq, K in dkdv) are copied once into TMEM by the softmax warps,
 // so those N = 64 products read only the streamed 64-row tile from shared
 // memory: shared-memory bandwidth, not the tensor core, bounded them when A
-// came from shared memory too.
+// came from shared memory too. (Writing dS to a TMEM area of its own, so the
+// next scores need not wait for the dQ product, measured 14% slower: it left no
+// TMEM for the operands above, and the products they feed went back to
+// reading both operands from shared memory.)
 // Every mbarrier wait is bounded; on expiry the kernel records an error code,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -44,8 +51,17 @@ using namespace ptx;
 
 constexpr int BM = 128;  // rows owned by a CTA (queries for dq, keys for dkdv)
 constexpr int BN = 64;   // streamed tile width (keys for dq, queries for dkdv)
-constexpr int kSoftmaxWarps = 8;
+constexpr int kGroups = 2;                  // softmax warpgroups
+constexpr int kCols = BN / kGroups;         // tile columns per warpgroup
+constexpr int kSoftmaxWarps = 4 * kGroups;
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
+constexpr uint32_t kColMask = kCols == 32 ? 0xffffffffu : (1u << kCols) - 1u;
+
+// TMEM column offset of the packed bf16 pairs of tile columns [16 kk, 16 kk + 16)
+// inside a buffer, when warpgroup g packs its kCols columns at g * kCols.
+__host__ __device__ constexpr uint32_t packed_col(int kk) {
+  return uint32_t((16 * kk / kCols) * kCols + (16 * kk % kCols) / 2);
+}
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __noinline__ void bwd_raise(volatile int *abort_flag, uint32_t code) {
@@ -92,13 +108,34 @@ __device__ __forceinline__ uint32_t bits_in(int32_t lo, int32_t hi) {
   return uint32_t(((1ull << hi) - 1ull) & ~((1ull << lo) - 1ull));
 }
 
-// Tile index of the j-th visited tile of up to three ascending ranges.
-__device__ __forceinline__ int32_t nth_tile(int32_t j, const int32_t (&t)[6]) {
-  const int32_t n0 = t[1] - t[0], n1 = t[3] - t[2];
-  if (j < n0) return t[0] + j;
-  if (j < n0 + n1) return t[2] + (j - n0);
-  return t[4] + (j - n0 - n1);
+// Up to three ascending tile ranges, held in registers (the schedule functions
+// fill an array with computed indices, which would otherwise live in local
+// memory and be re-read for every tile).
+struct TileRanges {
+  int32_t s0, n0, s1, n1, s2;  // starts of the ranges; lengths of the first two
+  __device__ __forceinline__ explicit TileRanges(const int32_t (&t)[6])
+      : s0(t[0]), n0(t[1] - t[0]), s1(t[2]), n1(t[3] - t[2]), s2(t[4]) {}
+};
+
+// Tile index of the j-th visited tile.
+__device__ __forceinline__ int32_t nth_tile(int32_t j, const TileRanges &r) {
+  if (j < r.n0) return r.s0 + j;
+  if (j < r.n0 + r.n1) return r.s1 + (j - r.n0);
+  return r.s2 + (j - r.n0 - r.n1);
 }
+
+// TMEM accesses of 8, 16 or 32 columns, chosen by the register array's size.
+__device__ __forceinline__ void tmem_ld_pair(uint32_t a, uint32_t b, uint32_t (&x)[16], uint32_t (&y)[16]) {
+  tmem_ld16x2(a, b, x, y);
+}
+__device__ __forceinline__ void tmem_ld_pair(uint32_t a, uint32_t b, uint32_t (&x)[32], uint32_t (&y)[32]) {
+  tmem_ld32x2(a, b, x, y);
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t a, uint32_t (&x)[16]) { tmem_ld16(a, x); }
+__device__ __forceinline__ void tmem_ld_cols(uint32_t a, uint32_t (&x)[32]) { tmem_ld32(a, x); }
+__device__ __forceinline__ void tmem_st_cols(uint32_t a, const uint32_t (&x)[8]) { tmem_st8(a, x); }
+__device__ __forceinline__ void tmem_st_cols(uint32_t a, const uint32_t (&x)[16]) { tmem_st16(a, x); }
+__device__ __forceinline__ void tmem_st_cols(uint32_t a, const uint32_t (&x)[32]) { tmem_st32(a, x); }
 
 // NRES: resident 128-row tiles kept in shared memory (0 in dq, V in dkdv).
 template <int D, int NRES>
@@ -143,13 +180,14 @@ __device__ __forceinline__ BBars bbars(uint32_t base) {
   return b;
 }
 
-// Copies half g of this thread's bf16 row into TMEM as packed pairs: column
-// taddr + i holds elements (2i, 2i+1) of the row, the layout in which the
-// tensor core reads an A operand from TMEM (one 16-element K step per 8
-// columns). Rows past the sequence are zero, as a TMA copy would fill them.
+// Copies part g (of kGroups) of this thread's bf16 row into TMEM as packed
+// pairs: column taddr + i holds elements (2i, 2i+1) of the row, the layout in
+// which the tensor core reads an A operand from TMEM (one 16-element K step per
+// 8 columns). Rows past the sequence are zero, as a TMA copy would fill them.
 template <int D>
 __device__ __forceinline__ void row_to_tmem(const uint16_t *row, bool live, uint32_t taddr, int g) {
-  constexpr int W = D / 4;  // 32-bit words in half a row
+  constexpr int W = D / (2 * kGroups);  // 32-bit words in one part of a row
+  static_assert(W % 4 == 0 && W >= 8, "row part must be whole 16-byte loads and >= 8 columns");
   uint32_t w[W];
   const uint4 *s4 = reinterpret_cast<const uint4 *>(row) + g * (W / 4);
 #pragma unroll
@@ -160,11 +198,7 @@ __device__ __forceinline__ void row_to_tmem(const uint16_t *row, bool live, uint
     w[4 * v + 2] = x.z;
     w[4 * v + 3] = x.w;
   }
-  if constexpr (W == 32) {
-    tmem_st32(taddr + g * W, w);
-  } else {
-    tmem_st16(taddr + g * W, w);
-  }
+  tmem_st_cols(taddr + g * W, w);
 }
 
 // Shared prologue of both kernels: barriers, TMEM, error checks. Returns false
@@ -219,9 +253,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
   const int32_t bh = blockIdx.x / p.n_row_tiles;
   const int32_t qt = p.row_order[blockIdx.x % p.n_row_tiles];
   const int32_t q0 = qt * BM, q1 = min(q0 + BM, p.geom.N);
-  int32_t t[6];
-  const int32_t ntiles = qtile_key_tiles(p.geom, q0, q1, BN, t[0], t[1], t[2], t[3]);
-  t[4] = t[5] = t[3];
+  int32_t tr[6];
+  const int32_t ntiles = qtile_key_tiles(p.geom, q0, q1, BN, tr[0], tr[1], tr[2], tr[3]);
+  tr[4] = tr[5] = tr[3];
+  const TileRanges t(tr);
 
   bwd_setup<C>(sbase, sgen, bar, warp);
   const uint32_t tmem = *tmem_slot;
@@ -286,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
         const uint32_t aS = tmem + COL_S0 + (i & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;  // packed dS columns of keys 16kk..
+          const uint32_t pc = packed_col(kk);  // packed dS columns of keys 16kk..
           mma_ts(leader, tmem, aS + pc, dKmn0 + so + uint64_t((kk * 16 * 128) >> 4), ID_Q,
                  (i > 0 || kk > 0) ? 1u : 0u);
         }
@@ -329,27 +364,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
         break;
       }
       tc_fence_after();
-      const int32_t kh = nth_tile(j, t) * BN + 32 * g;
-      const uint32_t cS = lane_addr + COL_S0 + b * 128 + 32 * g;
-      uint32_t rs[32], rp[32];
-      tmem_ld32x2(cS, cS + 64, rs, rp);
-      const uint32_t vis = bits_in(a0 - kh, b0 - kh) | bits_in(a1 - kh, b1 - kh);
-      if (vis != 0xffffffffu) {  // hidden keys: p = 0 and no dP (select, NaN-safe)
+      const int32_t kh = nth_tile(j, t) * BN + kCols * g;
+      const uint32_t cS = lane_addr + COL_S0 + b * 128 + kCols * g;
+      uint32_t rs[kCols], rp[kCols];
+      tmem_ld_pair(cS, cS + 64, rs, rp);
+      const uint32_t vis = (bits_in(a0 - kh, b0 - kh) | bits_in(a1 - kh, b1 - kh)) & kColMask;
+      if (vis != kColMask) {  // hidden keys: p = 0 and no dP (select, NaN-safe)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < kCols; ++i) {
           const bool v = (vis >> i) & 1u;
           rs[i] = v ? rs[i] : __float_as_uint(-INFINITY);
           rp[i] = v ? rp[i] : __float_as_uint(dl);
         }
       }
-      uint32_t pk[16];
+      uint32_t pk[kCols / 2];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < kCols / 2; ++i) {
         const float pa = ex2(fmaf(__uint_as_float(rs[2 * i]), sl2, -lse2));
         const float pb = ex2(fmaf(__uint_as_float(rs[2 * i + 1]), sl2, -lse2));
         pk[i] = pack_bf16(pa * (__uint_as_float(rp[2 * i]) - dl), pb * (__uint_as_float(rp[2 * i + 1]) - dl));
       }
-      tmem_st16(cS, pk);
+      tmem_st_cols(cS, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -360,17 +395,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       if (bwarp_wait(bar.o_done + 8 * (last & 1), (last >> 1) & 1, abort_flag, p.timeout_ns, 26)) {
         tc_fence_after();
         uint4 *out = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.dq) + ri * D);
+        constexpr int GC = D / kGroups, EC = GC < 32 ? GC : 32;  // columns per group, per load
 #pragma unroll 1
-        for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + c, r);
-          uint32_t po[16];
+        for (int c = g * GC; c < (g + 1) * GC; c += EC) {
+          uint32_t r[EC];
+          tmem_ld_cols(lane_addr + c, r);
+          uint32_t po[EC / 2];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < EC / 2; ++i)
             po[i] = pack_bf16(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
           if (live) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
+            for (int v = 0; v < EC / 8; ++v)
               out[c / 8 + v] = make_uint4(po[4 * v], po[4 * v + 1], po[4 * v + 2], po[4 * v + 3]);
           }
         }
@@ -404,8 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
   const int32_t bh = blockIdx.x / p.n_row_tiles;
   const int32_t kt = p.row_order[blockIdx.x % p.n_row_tiles];
   const int32_t k0 = kt * BM, k1 = min(k0 + BM, p.geom.N);
-  int32_t t[6];
-  const int32_t ntiles = ktile_query_tiles(p.geom, k0, k1, BN, t);
+  int32_t tr[6];
+  const int32_t ntiles = ktile_query_tiles(p.geom, k0, k1, BN, tr);
+  const TileRanges t(tr);
 
   bwd_setup<C>(sbase, sgen, bar, warp);
   const uint32_t tmem = *tmem_slot;
@@ -499,12 +536,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         const uint32_t aP = tmem + COL_S0 + (i & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // queries 16kk.. : warpgroup kk>>1 packed P^T at +0 and dS^T at +16 of its 32 columns
-          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;
+          // queries 16kk..: packed P^T in the first half of its warpgroup's
+          // columns, dS^T in the second half
+          const uint32_t pc = packed_col(kk);
           const uint64_t ko = uint64_t((kk * 16 * 128) >> 4);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
           mma_ts(leader, tmem, aP + pc, dOmn0 + so + ko, ID_A, acc);           // dV += P^T dO
-          mma_ts(leader, tmem + D, aP + 16 + pc, dQmn0 + so + ko, ID_A, acc);  // dK += dS^T Q
+          mma_ts(leader, tmem + D, aP + kCols / 2 + pc, dQmn0 + so + ko, ID_A, acc);  // dK += dS^T Q
         }
         tc_commit(leader, bar.o_done + 8 * (i & 1));
         tc_commit(leader, bar.st_empty + 8 * s);
@@ -538,27 +576,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         break;
       }
       tc_fence_after();
-      const int32_t qh = nth_tile(j, t) * BN + 32 * g;
-      const uint32_t cS = lane_addr + COL_S0 + b * 64 + 32 * g;
-      uint32_t rs[32], rp[32];
-      tmem_ld32x2(cS, lane_addr + COL_DP + 32 * g, rs, rp);
+      const int32_t qh = nth_tile(j, t) * BN + kCols * g;
+      const uint32_t cS = lane_addr + COL_S0 + b * 64 + kCols * g;
+      uint32_t rs[kCols], rp[kCols];
+      tmem_ld_pair(cS, lane_addr + COL_DP + kCols * g, rs, rp);
       tc_fence_before();  // dP^T is in registers: its buffer may be overwritten
       __syncwarp();
       if (lane == 0) mbar_arrive(bar.dp_free);
-      const uint32_t vis = bits_in(a0 - qh, b0 - qh) | bits_in(a1 - qh, b1 - qh);
-      if (vis != 0xffffffffu) {  // queries that do not see this key: p = 0, no dP
+      const uint32_t vis = (bits_in(a0 - qh, b0 - qh) | bits_in(a1 - qh, b1 - qh)) & kColMask;
+      if (vis != kColMask) {  // queries that do not see this key: p = 0, no dP
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < kCols; ++i) {
           const bool v = (vis >> i) & 1u;
           rs[i] = v ? rs[i] : __float_as_uint(-INFINITY);
           rp[i] = v ? rp[i] : 0u;
         }
       }
       const float4 *st4 = reinterpret_cast<const float4 *>(sgen + C::OFF_ST + s * C::STAGE +
-                                                           2 * C::S_BYTES) + 8 * g;
-      uint32_t pk[16], dk[16];
+                                                           2 * C::S_BYTES) + (kCols / 4) * g;
+      uint32_t pk[kCols / 2], dk[kCols / 2];
 #pragma unroll
-      for (int i4 = 0; i4 < 8; ++i4) {
+      for (int i4 = 0; i4 < kCols / 4; ++i4) {
         const float4 l4 = st4[i4], d4 = st4[16 + i4];
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
@@ -573,8 +611,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
           dk[i] = pack_bf16(pa * da, pb * db);
         }
       }
-      tmem_st16(cS, pk);
-      tmem_st16(cS + 16, dk);
+      tmem_st_cols(cS, pk);
+      tmem_st_cols(cS + kCols / 2, dk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -587,19 +625,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         tc_fence_after();
         uint4 *odv = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.dv) + ri * D);
         uint4 *odk = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.dk) + ri * D);
+        constexpr int GC = D / kGroups, EC = GC < 32 ? GC : 32;  // columns per group, per load
 #pragma unroll 1
-        for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
-          uint32_t rv[32], rk[32];
-          tmem_ld32x2(lane_addr + c, lane_addr + D + c, rv, rk);
-          uint32_t pv[16], pkk[16];
+        for (int c = g * GC; c < (g + 1) * GC; c += EC) {
+          uint32_t rv[EC], rk[EC];
+          tmem_ld_pair(lane_addr + c, lane_addr + D + c, rv, rk);
+          uint32_t pv[EC / 2], pkk[EC / 2];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < EC / 2; ++i) {
             pv[i] = pack_bf16(__uint_as_float(rv[2 * i]), __uint_as_float(rv[2 * i + 1]));
             pkk[i] = pack_bf16(__uint_as_float(rk[2 * i]) * p.scale, __uint_as_float(rk[2 * i + 1]) * p.scale);
           }
           if (live) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
+            for (int v = 0; v < EC / 8; ++v) {
               odv[c / 8 + v] = make_uint4(pv[4 * v], pv[4 * v + 1], pv[4 * v + 2], pv[4 * v + 3]);
               odk[c / 8 + v] = make_uint4(pkk[4 * v], pkk[4 * v + 1], pkk[4 * v + 2], pkk[4 * v + 3]);
             }
@@ -610,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       // a key no query sees (cannot happen for valid masks): zero gradients
       uint4 *odv = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.dv) + ri * D);
       uint4 *odk = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.dk) + ri * D);
-      for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 8) {
+      for (int c = g * (D / kGroups); c < (g + 1) * (D / kGroups); c += 8) {
         odv[c / 8] = make_uint4(0, 0, 0, 0);
         odk[c / 8] = make_uint4(0, 0, 0, 0);
       }
