@@ -29,6 +29,7 @@
 #ifndef CAUSALJVP_H
 #define CAUSALJVP_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -102,6 +103,36 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v,
                             const caj_problem *prob, const caj_mask_desc *mask,
                             void *o, void *to, float *lse, float *tlse,
                             void *stream);
+
+/*
+ * Host-buffer form of caj_attn_fwd_jvp: the same operation, with the inputs
+ * and outputs in host memory. The heads are split into at most 16 chunks.
+ * Three things run at once on three streams: the copy of chunk c's six inputs
+ * to the device, the kernel on chunk c-1, and the copy of an earlier chunk's
+ * outputs back to the host. Pinned host memory lets the copies overlap;
+ * pageable memory gives the same results, but its copies do not overlap.
+ *   in : q, k, v, tq, tk, tv   host, [B,H,N,D] of prob->dtype, read only
+ *   out: o, to                 host, [B,H,N,D] of prob->dtype
+ *        lse, tlse             host, [B,H,N] fp32
+ *   workspace                  device memory, 256-byte aligned, of at least
+ *                              caj_attn_fwd_jvp_host_workspace() bytes. It is
+ *                              owned by the caller and not freed here. No other
+ *                              work may use it until the call has completed.
+ *   stream                     the call runs after the work already on
+ *                              `stream`. The outputs are complete in host
+ *                              memory once `stream` has passed the call, e.g.
+ *                              after cudaStreamSynchronize(stream).
+ * The library keeps two copy streams and a set of events per device, created
+ * on first use. Returns as caj_attn_fwd_jvp, and CAJ_ERR_INVALID_ARG also
+ * for a null, misaligned or too small workspace. After a failure, `stream`
+ * still waits for every copy the call enqueued.
+ */
+caj_status caj_attn_fwd_jvp_host_workspace(const caj_problem *prob, size_t *bytes);
+caj_status caj_attn_fwd_jvp_host(const void *q, const void *k, const void *v,
+                                 const void *tq, const void *tk, const void *tv,
+                                 const caj_problem *prob, const caj_mask_desc *mask,
+                                 void *o, void *to, float *lse, float *tlse,
+                                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Attention-block prologue in primal-tangent form. Causal-rCM implements the

@@ -8,8 +8,9 @@ q..tv are [B, H, N, D] tensors (bf16 for the tensor-core path, fp32 for the
 CUDA-core fp32 path), `mask` a MaskDesc (or a (tokens_per_frame,
 frames_per_chunk, n_frames, tf_layout) tuple). With CUDA tensors everything
 stays on the device and the call is asynchronous on the current stream. With
-CPU tensors the inputs are copied to the current CUDA device and the outputs
-copied back (the end-to-end path).
+CPU tensors the library's host-buffer entry point copies the inputs to the
+current CUDA device and the outputs back, overlapping the copies with the
+kernels chunk by chunk (the end-to-end path).
 
 The operation is the masked FlashAttention JVP of the Causal-rCM paper
 (appendix B, eq. 42-45): O = softmax(scale Q K^T + M) V,
@@ -111,27 +112,45 @@ def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optiona
 
 def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
                  clean_tangent_zero: bool = False):
-    """Returns (o, to, lse, tlse). See the module docstring and attn_fwd_jvp_out."""
-    host = not q.is_cuda
-    if host:
-        dev = torch.device("cuda", torch.cuda.current_device())
-        ins = [t.to(dev, non_blocking=True) for t in (q, k, v, tq, tk, tv)]
-    else:
+    """Returns (o, to, lse, tlse). See the module docstring and attn_fwd_jvp_out.
+
+    With CPU tensors the library's host-buffer entry point runs the call: it
+    copies head chunks to a device workspace, runs the kernel on each chunk and
+    copies the outputs back, with the three overlapped. Outputs are returned
+    in pinned host memory; pinned inputs copy fastest."""
+    if q.is_cuda:
         ins = [q, k, v, tq, tk, tv]
-    q_ = ins[0]
-    o = torch.empty_like(q_)
-    to = torch.empty_like(q_)
-    lse = torch.empty(q_.shape[:3], dtype=torch.float32, device=q_.device)
-    tlse = torch.empty_like(lse)
-    attn_fwd_jvp_out(*ins, mask, o, to, lse, tlse, scale=scale, clean_tangent_zero=clean_tangent_zero)
-    if host:
-        outs = []
-        for t in (o, to, lse, tlse):
-            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-            h.copy_(t, non_blocking=True)
-            outs.append(h)
-        torch.cuda.current_stream().synchronize()
-        return tuple(outs)
+        o = torch.empty_like(q)
+        to = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        tlse = torch.empty_like(lse)
+        attn_fwd_jvp_out(*ins, mask, o, to, lse, tlse, scale=scale, clean_tangent_zero=clean_tangent_zero)
+        return o, to, lse, tlse
+    ins = (q, k, v, tq, tk, tv)
+    for t in ins:
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("attn_fwd_jvp: host inputs must be contiguous CPU tensors")
+    if q.dtype not in _DTYPES or any(t.dtype != q.dtype or t.shape != q.shape for t in ins):
+        raise ValueError("attn_fwd_jvp: q..tv must share one shape and dtype (bf16 or fp32)")
+    prob = _problem(q, scale, clean_tangent_zero)
+    L = _lib.lib()
+    nbytes = ctypes.c_size_t(0)
+    _lib.check(L.caj_attn_fwd_jvp_host_workspace(ctypes.byref(prob), ctypes.byref(nbytes)),
+               "caj_attn_fwd_jvp_host_workspace")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=dev)
+    o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    to = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)
+    tlse = torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)
+    stream = torch.cuda.current_stream(dev)
+    st = L.caj_attn_fwd_jvp_host(*[ctypes.c_void_p(t.data_ptr()) for t in ins], ctypes.byref(prob),
+                                 ctypes.byref(_lib.mask_c(mask)),
+                                 *[ctypes.c_void_p(t.data_ptr()) for t in (o, to, lse, tlse)],
+                                 ctypes.c_void_p(workspace.data_ptr()), nbytes,
+                                 ctypes.c_void_p(stream.cuda_stream))
+    _lib.check(st, "caj_attn_fwd_jvp_host")
+    stream.synchronize()
     return o, to, lse, tlse
 
 

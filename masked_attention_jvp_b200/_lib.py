@@ -17,7 +17,7 @@ EXPORTED = [
     "caj_status_string", "caj_last_cuda_error", "caj_validate_mask", "caj_visible_pairs",
     "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
     "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
-    "caj_attn_bwd",
+    "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host",
 ]
 
 
@@ -91,6 +91,11 @@ def lib() -> ctypes.CDLL:
         L.caj_ktile_query_tiles.restype = i32
         L.caj_attn_bwd.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC)] + [vp] * 5
         L.caj_attn_bwd.restype = ctypes.c_int
+        L.caj_attn_fwd_jvp_host_workspace.argtypes = [ctypes.POINTER(ProblemC), ctypes.POINTER(ctypes.c_size_t)]
+        L.caj_attn_fwd_jvp_host_workspace.restype = ctypes.c_int
+        L.caj_attn_fwd_jvp_host.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC)] + \
+            [vp] * 5 + [ctypes.c_size_t, vp]
+        L.caj_attn_fwd_jvp_host.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

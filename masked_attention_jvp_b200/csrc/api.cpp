@@ -120,6 +120,84 @@ uint64_t wait_timeout_ns() {
 
 }  // namespace
 
+namespace {
+
+// Shape, dtype, flag and mask checks shared by the device and host forms of
+// the forward.
+caj_status validate_fwd(const caj_problem *prob, const caj_mask_desc *mask, caj::MaskGeom *g) {
+  if (!prob || !mask) return CAJ_ERR_INVALID_ARG;
+  if (prob->B <= 0 || prob->H <= 0 || prob->N <= 0 || prob->D <= 0) return CAJ_ERR_INVALID_ARG;
+  if (!geom_from_desc(mask, g) || g->N != prob->N) return CAJ_ERR_INVALID_ARG;
+  if (prob->dtype != CAJ_DTYPE_F32 && prob->dtype != CAJ_DTYPE_BF16) return CAJ_ERR_INVALID_ARG;
+  if (!(prob->scale >= 0.f) || std::isinf(prob->scale)) return CAJ_ERR_INVALID_ARG;
+  if (prob->flags & ~int32_t(CAJ_FLAG_CLEAN_TANGENT_ZERO)) return CAJ_ERR_INVALID_ARG;
+  if ((prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) && !mask->tf_layout) return CAJ_ERR_INVALID_ARG;
+  if (prob->D != 64 && prob->D != 128) return CAJ_ERR_UNSUPPORTED;
+  const int64_t BH = int64_t(prob->B) * prob->H;
+  if (BH > 65535 || prob->N > (1 << 20)) return CAJ_ERR_UNSUPPORTED;
+  return CAJ_OK;
+}
+
+// Device workspace of the host-buffer forward: the six inputs, O, tO, LSE and
+// tLSE, each region 256-byte aligned.
+struct HostWorkspace {
+  size_t in[6], o, to, lse, tlse, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool host_workspace(const caj_problem *prob, HostWorkspace *w) {
+  if (!prob || prob->B <= 0 || prob->H <= 0 || prob->N <= 0 || prob->D <= 0) return false;
+  const size_t es = prob->dtype == CAJ_DTYPE_BF16 ? 2 : prob->dtype == CAJ_DTYPE_F32 ? 4 : 0;
+  if (!es) return false;
+  const size_t rows = size_t(prob->B) * size_t(prob->H) * size_t(prob->N);
+  const size_t tensor = align256(rows * size_t(prob->D) * es), stats = align256(rows * 4);
+  size_t off = 0;
+  for (int i = 0; i < 6; ++i, off += tensor) w->in[i] = off;
+  w->o = off;
+  off += tensor;
+  w->to = off;
+  off += tensor;
+  w->lse = off;
+  off += stats;
+  w->tlse = off;
+  off += stats;
+  w->total = off;
+  return true;
+}
+
+// Copy streams and events of the host-buffer forward, one set per device,
+// created on first use and kept for the life of the process.
+constexpr int kHostChunks = 16;  // at most this many head chunks per call
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in_ready[kHostChunks] = {}, out_ready[kHostChunks] = {};
+};
+std::mutex g_pipe_mu;
+std::vector<std::unique_ptr<HostPipe>> g_pipes;
+
+cudaError_t host_pipe(int dev, HostPipe **out) {
+  if (int(g_pipes.size()) <= dev) g_pipes.resize(dev + 1);
+  if (!g_pipes[dev]) {
+    std::unique_ptr<HostPipe> p(new HostPipe());
+    cudaError_t e = cudaStreamCreateWithFlags(&p->in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->start, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->done, cudaEventDisableTiming);
+    for (int c = 0; c < kHostChunks && e == cudaSuccess; ++c) {
+      e = cudaEventCreateWithFlags(&p->in_ready[c], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->out_ready[c], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return e;  // the partial set is not kept; nothing was enqueued
+    g_pipes[dev] = std::move(p);
+  }
+  *out = g_pipes[dev].get();
+  return cudaSuccess;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *caj_status_string(caj_status s) {
@@ -196,24 +274,17 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
                             const void *tk, const void *tv, const caj_problem *prob,
                             const caj_mask_desc *mask, void *o, void *to, float *lse, float *tlse,
                             void *stream) {
-  if (!prob || !mask) return CAJ_ERR_INVALID_ARG;
   const void *ins[6] = {q, k, v, tq, tk, tv};
   for (const void *p : ins)
     if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
   if (!o || !to || !aligned16(o) || !aligned16(to)) return CAJ_ERR_INVALID_ARG;
   if (!lse || !tlse || !aligned4(lse) || !aligned4(tlse)) return CAJ_ERR_INVALID_ARG;
-  if (prob->B <= 0 || prob->H <= 0 || prob->N <= 0 || prob->D <= 0) return CAJ_ERR_INVALID_ARG;
   caj::MaskGeom g;
-  if (!geom_from_desc(mask, &g) || g.N != prob->N) return CAJ_ERR_INVALID_ARG;
-  if (prob->dtype != CAJ_DTYPE_F32 && prob->dtype != CAJ_DTYPE_BF16) return CAJ_ERR_INVALID_ARG;
-  if (!(prob->scale >= 0.f) || std::isinf(prob->scale)) return CAJ_ERR_INVALID_ARG;
-  if (prob->flags & ~int32_t(CAJ_FLAG_CLEAN_TANGENT_ZERO)) return CAJ_ERR_INVALID_ARG;
-  if ((prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) && !mask->tf_layout) return CAJ_ERR_INVALID_ARG;
-  if (prob->D != 64 && prob->D != 128) return CAJ_ERR_UNSUPPORTED;
+  caj_status st = validate_fwd(prob, mask, &g);
+  if (st != CAJ_OK) return st;
   const int64_t BH = int64_t(prob->B) * prob->H;
-  if (BH > 65535 || prob->N > (1 << 20)) return CAJ_ERR_UNSUPPORTED;
 
-  caj_status st = check_device();
+  st = check_device();
   if (st != CAJ_OK) return st;
 
   const float scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt(float(prob->D));
@@ -269,6 +340,90 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
 
   cudaError_t e = caj::launch_fwd_jvp_sm100(p, D, s);
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+}
+
+caj_status caj_attn_fwd_jvp_host_workspace(const caj_problem *prob, size_t *bytes) {
+  HostWorkspace w;
+  if (!bytes || !host_workspace(prob, &w)) return CAJ_ERR_INVALID_ARG;
+  *bytes = w.total;
+  return CAJ_OK;
+}
+
+caj_status caj_attn_fwd_jvp_host(const void *q, const void *k, const void *v, const void *tq,
+                                 const void *tk, const void *tv, const caj_problem *prob,
+                                 const caj_mask_desc *mask, void *o, void *to, float *lse,
+                                 float *tlse, void *workspace, size_t workspace_bytes,
+                                 void *stream) {
+  const void *hin[6] = {q, k, v, tq, tk, tv};
+  for (const void *p : hin)
+    if (!p) return CAJ_ERR_INVALID_ARG;
+  if (!o || !to || !lse || !tlse) return CAJ_ERR_INVALID_ARG;
+  caj::MaskGeom g;
+  caj_status st = validate_fwd(prob, mask, &g);
+  if (st != CAJ_OK) return st;
+  HostWorkspace w;
+  if (!host_workspace(prob, &w) || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < w.total)
+    return CAJ_ERR_INVALID_ARG;
+  st = check_device();
+  if (st != CAJ_OK) return st;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe *pp = nullptr;
+  if ((e = host_pipe(dev, &pp)) != cudaSuccess) return cuda_fail(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t es = prob->dtype == CAJ_DTYPE_BF16 ? 2 : 4;
+  const int64_t BH = int64_t(prob->B) * prob->H;
+  const int64_t hpc = (BH + kHostChunks - 1) / kHostChunks;  // heads per chunk
+  const int64_t nchunks = (BH + hpc - 1) / hpc;
+  const size_t head_elems = size_t(prob->N) * size_t(prob->D), head_rows = size_t(prob->N);
+
+  // Both copy streams start after the work already on `stream` (an earlier
+  // call may still read this workspace), and `stream` ends after both.
+  auto ok = [&](cudaError_t r) { return r == cudaSuccess || (e = r, false); };
+  bool good = ok(cudaEventRecord(pp->start, s)) && ok(cudaStreamWaitEvent(pp->in, pp->start, 0)) &&
+              ok(cudaStreamWaitEvent(pp->out, pp->start, 0));
+  caj_status kst = CAJ_OK;
+  for (int64_t c = 0; good && c < nchunks; ++c) {
+    const int64_t h0 = c * hpc, nh = std::min(hpc, BH - h0);
+    const size_t off = size_t(h0) * head_elems * es, bytes = size_t(nh) * head_elems * es;
+    const size_t soff = size_t(h0) * head_rows * 4, sbytes = size_t(nh) * head_rows * 4;
+    for (int i = 0; good && i < 6; ++i)
+      good = ok(cudaMemcpyAsync(ws + w.in[i] + off, static_cast<const uint8_t *>(hin[i]) + off, bytes,
+                                cudaMemcpyHostToDevice, pp->in));
+    good = good && ok(cudaEventRecord(pp->in_ready[c], pp->in)) &&
+           ok(cudaStreamWaitEvent(s, pp->in_ready[c], 0));
+    if (!good) break;
+    // the chunk's heads form a problem of their own: [1, nh, N, D] at offset h0
+    caj_problem sub = *prob;
+    sub.B = 1;
+    sub.H = int32_t(nh);
+    kst = caj_attn_fwd_jvp(ws + w.in[0] + off, ws + w.in[1] + off, ws + w.in[2] + off,
+                           ws + w.in[3] + off, ws + w.in[4] + off, ws + w.in[5] + off, &sub, mask,
+                           ws + w.o + off, ws + w.to + off, reinterpret_cast<float *>(ws + w.lse + soff),
+                           reinterpret_cast<float *>(ws + w.tlse + soff), stream);
+    if (kst != CAJ_OK) break;
+    good = ok(cudaEventRecord(pp->out_ready[c], s)) && ok(cudaStreamWaitEvent(pp->out, pp->out_ready[c], 0)) &&
+           ok(cudaMemcpyAsync(static_cast<uint8_t *>(o) + off, ws + w.o + off, bytes, cudaMemcpyDeviceToHost, pp->out)) &&
+           ok(cudaMemcpyAsync(static_cast<uint8_t *>(to) + off, ws + w.to + off, bytes, cudaMemcpyDeviceToHost, pp->out)) &&
+           ok(cudaMemcpyAsync(reinterpret_cast<uint8_t *>(lse) + soff, ws + w.lse + soff, sbytes,
+                              cudaMemcpyDeviceToHost, pp->out)) &&
+           ok(cudaMemcpyAsync(reinterpret_cast<uint8_t *>(tlse) + soff, ws + w.tlse + soff, sbytes,
+                              cudaMemcpyDeviceToHost, pp->out));
+  }
+  // Join both copy streams back into `stream`, also after a failure, so that no
+  // copy touches the caller's buffers once `stream` has passed this call.
+  cudaError_t je = cudaEventRecord(pp->done, pp->in);
+  if (je == cudaSuccess) je = cudaStreamWaitEvent(s, pp->done, 0);
+  if (je == cudaSuccess) je = cudaEventRecord(pp->done, pp->out);
+  if (je == cudaSuccess) je = cudaStreamWaitEvent(s, pp->done, 0);
+  if (kst != CAJ_OK) return kst;
+  if (!good) return cuda_fail(e);
+  return je == cudaSuccess ? CAJ_OK : cuda_fail(je);
 }
 
 caj_status caj_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv, const void *txq,

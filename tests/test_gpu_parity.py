@@ -172,15 +172,50 @@ def test_outputs_fully_overwritten(dtype):
         assert torch.isfinite(t).all()
 
 
-def test_host_tensor_path_matches_device_path():
-    w = Workload("host", 1, 2, 128, MaskDesc(90, 1, 4, 1), torch.bfloat16, seed=12)
+# (mask, B, H, D, dtype, pinned, clean_tangent_zero): head counts that fill 16
+# chunks of one head, 14 chunks of 3 heads with a short last chunk, and one head
+HOST = [(MaskDesc(90, 1, 4, 1), 1, 2, 128, torch.bfloat16, True, False),
+        (MaskDesc(33, 2, 4, 0), 1, 13, 64, torch.bfloat16, True, False),
+        (MaskDesc(20, 1, 3, 1), 4, 10, 128, torch.bfloat16, False, False),
+        (MaskDesc(45, 2, 4, 1), 1, 3, 128, torch.bfloat16, True, True),
+        (MaskDesc(17, 1, 3, 0), 1, 1, 64, torch.float32, True, False)]
+
+
+@pytest.mark.parametrize("case", range(len(HOST)))
+def test_host_entry_matches_device_path(case):
+    """The host-buffer entry point (chunked copies overlapped with the kernels)
+    gives bitwise the device path's results."""
+    mask, B, H, D, dtype, pinned, ctz = HOST[case]
+    w = Workload(f"host{case}", B, H, D, mask, dtype, seed=12 + case)
     host = make_inputs(w, "cpu")
-    pinned = [t.pin_memory() for t in host]
-    a = caj.attn_fwd_jvp(*pinned, w.mask)
+    if ctz:
+        from masked_attention_jvp_b200.workloads import zero_clean_tangents
+        zero_clean_tangents(w, *host[3:])
+    if pinned:
+        host = [t.pin_memory() for t in host]
+    a = caj.attn_fwd_jvp(*host, w.mask, clean_tangent_zero=ctz)
     assert all(not t.is_cuda for t in a)
-    b = caj.attn_fwd_jvp(*[t.cuda() for t in host], w.mask)
+    b = caj.attn_fwd_jvp(*[t.cuda() for t in host], w.mask, clean_tangent_zero=ctz)
+    torch.cuda.synchronize()
+    caj.device_status()
     for x, y in zip(a, b):
         assert torch.equal(x, y.cpu())
+
+
+def test_host_entry_back_to_back_calls_reuse_nothing_stale():
+    """Two host calls in a row on different inputs: the second call's results
+    are its own (the copies of one call are ordered after the previous one)."""
+    w1 = Workload("hostA", 1, 4, 128, MaskDesc(64, 1, 4, 1), torch.bfloat16, seed=31)
+    w2 = Workload("hostB", 1, 4, 128, MaskDesc(64, 1, 4, 1), torch.bfloat16, seed=32)
+    h1 = [t.pin_memory() for t in make_inputs(w1, "cpu")]
+    h2 = [t.pin_memory() for t in make_inputs(w2, "cpu")]
+    a1 = caj.attn_fwd_jvp(*h1, w1.mask)
+    a2 = caj.attn_fwd_jvp(*h2, w2.mask)
+    b2 = caj.attn_fwd_jvp(*[t.cuda() for t in h2], w2.mask)
+    torch.cuda.synchronize()
+    for x, y in zip(a2, b2):
+        assert torch.equal(x, y.cpu())
+    assert not torch.equal(a1[0], a2[0])
 
 
 def test_rejects_mismatched_inputs_without_launch():

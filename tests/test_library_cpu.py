@@ -132,6 +132,50 @@ def test_argument_validation_launches_nothing():
     assert _call(prob=P(1, 2, 128, 64, bf, 0.0, 1), mask=M(16, 1, 4, 1)) != INV
 
 
+def _ws_bytes(prob):
+    n = ctypes.c_size_t(0)
+    st = _lib.lib().caj_attn_fwd_jvp_host_workspace(ctypes.byref(prob), ctypes.byref(n))
+    return st, n.value
+
+
+def test_host_workspace_size():
+    """Six inputs, O and tO of the problem's element size plus LSE and tLSE in
+    fp32, each region rounded up to 256 bytes."""
+    P = _lib.ProblemC
+    up = lambda x: (x + 255) // 256 * 256
+    for B, H, N, D, dt, es in [(1, 12, 65520, 128, _lib.CAJ_DTYPE_BF16, 2), (2, 3, 77, 64, _lib.CAJ_DTYPE_F32, 4),
+                               (1, 1, 1, 64, _lib.CAJ_DTYPE_BF16, 2)]:
+        st, n = _ws_bytes(P(B, H, N, D, dt, 0.0))
+        assert st == _lib.CAJ_OK
+        assert n == 8 * up(B * H * N * D * es) + 2 * up(B * H * N * 4)
+    assert _ws_bytes(P(1, 2, 64, 64, 7, 0.0))[0] == _lib.CAJ_ERR_INVALID_ARG   # unknown dtype
+    assert _ws_bytes(P(0, 2, 64, 64, 1, 0.0))[0] == _lib.CAJ_ERR_INVALID_ARG   # empty batch
+    n = ctypes.c_size_t(0)
+    assert _lib.lib().caj_attn_fwd_jvp_host_workspace(None, ctypes.byref(n)) == _lib.CAJ_ERR_INVALID_ARG
+
+
+def _host_call(workspace, nbytes, prob=None, mask=None, q=0x1000):
+    prob = prob or _lib.ProblemC(1, 2, 64, 64, _lib.CAJ_DTYPE_BF16, 0.0)
+    mask = mask or _lib.MaskDescC(16, 1, 4, 0)
+    vp = ctypes.c_void_p
+    return _lib.lib().caj_attn_fwd_jvp_host(vp(q), vp(q), vp(q), vp(q), vp(q), vp(q), ctypes.byref(prob),
+                                            ctypes.byref(mask), vp(q), vp(q), vp(q), vp(q),
+                                            vp(workspace), nbytes, vp(0))
+
+
+def test_host_entry_validation_copies_nothing():
+    """Bad arguments are refused before any copy is enqueued (these pointers are
+    never dereferenced)."""
+    INV, UNS = _lib.CAJ_ERR_INVALID_ARG, _lib.CAJ_ERR_UNSUPPORTED
+    _, need = _ws_bytes(_lib.ProblemC(1, 2, 64, 64, _lib.CAJ_DTYPE_BF16, 0.0))
+    assert _host_call(0, need) == INV                     # no workspace
+    assert _host_call(0x100080, need) == INV              # workspace not 256-byte aligned
+    assert _host_call(0x100000, need - 1) == INV          # workspace too small
+    assert _host_call(0x100000, need, q=0) == INV         # null input
+    assert _host_call(0x100000, need, mask=_lib.MaskDescC(16, 1, 5, 0)) == INV   # N != mask length
+    assert _host_call(0x100000, 1 << 40, prob=_lib.ProblemC(1, 2, 64, 96, _lib.CAJ_DTYPE_BF16, 0.0)) == UNS
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
 def test_valid_call_without_gpu_reports_cuda_error():
     assert _call() == _lib.CAJ_ERR_CUDA
