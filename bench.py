@@ -148,12 +148,58 @@ def time_oracle(w, target_s=15.0, host_inputs=None):
 
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    """SM clock and clock-event reasons of this process's GPU, sampled every
+    10 ms through NVML while the `with` block runs (reads only; nothing is set).
+    Falls back to `nvidia-smi -lms 100` where NVML is unavailable."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.01):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.rows = []          # (sm_mhz, max_mhz, reasons bitmask)
+        self.nvml = None
+        self.thread = None
+        self.stop = None
         self.proc = None
         self.path = None
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nvml = pynvml
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            pci = f"{getattr(props, 'pci_domain_id', 0):08x}:{bus:02x}:{getattr(props, 'pci_device_id', 0):02x}.0"
+            try:
+                return pynvml.nvmlDeviceGetHandleByPciBusId(pci)
+            except pynvml.NVMLError:
+                pass
+        return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def _sample(self, h):
+        nv = self.nvml
+        max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), max_mhz,
+                                  nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except nv.NVMLError:
+                return
+            self.stop.wait(self.period)
+
     def __enter__(self):
+        import threading
+        try:
+            h = self._nvml_handle()
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._sample, args=(h,), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -161,7 +207,7 @@ class ClockSampler:
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", f"--id={self.cuda_index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -169,32 +215,38 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            names = list(self.REASONS)
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    mask = sum(self.REASONS[n] for n, v in zip(names, parts[5:9]) if v == "Active")
+                    self.rows.append((float(parts[1]), float(parts[2]), mask))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
 
     def summary(self):
-        if self.proc is None or not self.path:
+        if not self.rows:
             return None
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted(n for n, bit in self.REASONS.items() if any(r[2] & bit for r in self.rows))
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": max(r[1] for r in self.rows),
+                "reasons": reasons, "samples": len(self.rows),
+                "source": "nvml, 10 ms" if self.nvml is not None else "nvidia-smi, 100 ms"}
 
 
 # ------------------------------------------------------------- multi-rank
