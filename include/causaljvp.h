@@ -185,12 +185,16 @@ caj_status caj_attn_bwd(const void *q, const void *k, const void *v, const void 
                         void *stream);
 
 /* Synchronises `stream`, then reads and clears the library's device error word.
- * Returns CAJ_OK, CAJ_ERR_DEVICE_TIMEOUT (a kernel abandoned a wait; its
- * outputs are undefined) or CAJ_ERR_CUDA. */
+ * Returns CAJ_OK, CAJ_ERR_DEVICE_TIMEOUT (a kernel gave up: it abandoned a wait
+ * or refused to run; its outputs are undefined) or CAJ_ERR_CUDA. */
 caj_status caj_last_device_status(void *stream);
 
-/* Detail of the last device error: which wait gave up (0 if none). Valid after
- * caj_last_device_status returned CAJ_ERR_DEVICE_TIMEOUT. */
+/* Detail of the last device error (0 if none). Valid after
+ * caj_last_device_status returned CAJ_ERR_DEVICE_TIMEOUT:
+ *   0x100 | site   a bounded wait expired at the numbered wait site;
+ *   0x200          the dynamic shared memory was not 1 KiB aligned;
+ *   0x300          a forward launch met a query tile of the other kind than it
+ *                  was built for (an internal partitioning error). */
 uint32_t caj_last_device_error_code(void);
 
 /* Sets the limit, in milliseconds, on every bounded wait inside the kernels of

@@ -325,7 +325,7 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   p.scale_log2e = scale * 1.4426950408889634f;
   p.timeout_ns = wait_timeout_ns();
   p.fault_mode = g_fault_mode.load();
-  p.clean_tangent_zero = (prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) ? 1 : 0;
+  p.tile_kind = caj::kTilesAll;
   // Launch order: query tiles by decreasing number of key tiles (ties: later first).
   std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
   for (int32_t t = 0; t < n_qtiles; ++t) {
@@ -336,6 +336,26 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   std::sort(cost.begin(), cost.end(), [](const auto &a, const auto &b) {
     return a.first != b.first ? a.first > b.first : a.second > b.second;
   });
+  if (prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) {
+    // Two launches, each over one kind of query tile in the same heaviest-first
+    // order: tiles with a noisy row (the dearer ones) first, then the clean ones.
+    std::unique_ptr<caj::Sm100Params> hc(new caj::Sm100Params(p));
+    int32_t nn = 0, nc = 0;
+    for (int32_t i = 0; i < n_qtiles; ++i) {
+      const int32_t t = cost[i].second;
+      if (std::min((t + 1) * caj::kBlockM, N) <= g.L)
+        hc->qtile_order[nc++] = uint16_t(t);
+      else
+        p.qtile_order[nn++] = uint16_t(t);
+    }
+    p.tile_kind = caj::kTilesNoisyCTZ;
+    p.n_qtiles = nn;
+    hc->tile_kind = caj::kTilesCleanCTZ;
+    hc->n_qtiles = nc;
+    cudaError_t e = nn ? caj::launch_fwd_jvp_sm100(p, D, s) : cudaSuccess;
+    if (e == cudaSuccess && nc) e = caj::launch_fwd_jvp_sm100(*hc, D, s);
+    return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+  }
   for (int32_t i = 0; i < n_qtiles; ++i) p.qtile_order[i] = uint16_t(cost[i].second);
 
   cudaError_t e = caj::launch_fwd_jvp_sm100(p, D, s);

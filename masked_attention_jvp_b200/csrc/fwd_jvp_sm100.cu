@@ -191,10 +191,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, timeout_ns, site));
 }
 
-// CTZ: clean-tangent-zero teacher forcing (the caller guarantees tq, tk, tv
-// vanish on rows < L); a separate instantiation so the dense kernel carries no
-// trace of the specialisation.
-template <int D, bool CTZ>
+// KIND (a TileKind): dense tangents, or one of the two kinds of query tile of
+// clean-tangent-zero teacher forcing (the caller guarantees tq, tk, tv vanish on
+// rows < L). Each is its own instantiation: the dense kernel carries no trace of
+// the specialisation, and neither CTZ kernel branches on its tiles' kind at run
+// time (measured: the branching kernel took 16.0 ms on the TF frame-wise
+// workload, the two specialised launches 11.7 ms).
+template <int D, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {
   using C = Cfg<D>;
@@ -223,8 +226,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t n0 = t1 - t0;
   // Clean-tangent-zero teacher forcing: a tile of clean query rows has no
   // tangent at all, and a key tile of clean tokens has tK = tV = 0.
-  const bool no_tan = CTZ && q1 <= p.geom.L;
+  constexpr bool CTZ = KIND != kTilesAll;
+  constexpr bool no_tan = KIND == kTilesCleanCTZ;  // clean query rows: primal only
   auto clean_keys = [&](int32_t key0) { return CTZ && key0 + BN <= p.geom.L; };
+  // The host partitions the query tiles by kind; a tile of the other kind is
+  // refused before any barrier or TMEM use (the whole CTA leaves together).
+  if (CTZ && (q1 <= p.geom.L) != no_tan) {
+    if (threadIdx.x == 0) atomicCAS(&g_device_error, 0u, uint32_t(kErrTileKind));
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q_full, 1);
@@ -618,28 +628,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CTZ>
+template <int D, int KIND>
 cudaError_t launch_impl(const Sm100Params &p, cudaStream_t stream) {
   using C = Cfg<D>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D, CTZ>,
+    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D, KIND>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
-  fwd_jvp_sm100_kernel<D, CTZ><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  fwd_jvp_sm100_kernel<D, KIND><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream) {
-  const bool ctz = p.clean_tangent_zero != 0;
-  if (D == 128) return ctz ? launch_impl<128, true>(p, stream) : launch_impl<128, false>(p, stream);
-  if (D == 64) return ctz ? launch_impl<64, true>(p, stream) : launch_impl<64, false>(p, stream);
-  return cudaErrorInvalidValue;
+  switch (p.tile_kind * 256 + D) {
+    case kTilesAll * 256 + 128: return launch_impl<128, kTilesAll>(p, stream);
+    case kTilesNoisyCTZ * 256 + 128: return launch_impl<128, kTilesNoisyCTZ>(p, stream);
+    case kTilesCleanCTZ * 256 + 128: return launch_impl<128, kTilesCleanCTZ>(p, stream);
+    case kTilesAll * 256 + 64: return launch_impl<64, kTilesAll>(p, stream);
+    case kTilesNoisyCTZ * 256 + 64: return launch_impl<64, kTilesNoisyCTZ>(p, stream);
+    case kTilesCleanCTZ * 256 + 64: return launch_impl<64, kTilesCleanCTZ>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, uint32_t *out) {

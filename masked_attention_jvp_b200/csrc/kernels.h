@@ -21,6 +21,17 @@ enum DeviceError : uint32_t {
   kErrNone = 0,
   kErrTimeoutBase = 0x100,     // | wait site
   kErrSmemMisaligned = 0x200,  // dynamic shared memory not 1 KiB aligned
+  kErrTileKind = 0x300,        // a query tile outside the kind its launch covers
+};
+
+// Query tiles of one launch of the tensor-core forward. With clean-tangent-zero
+// teacher forcing (tq, tk, tv vanish on rows < L) a call runs as two launches,
+// one per kind of query tile: each kernel instantiation carries only its own
+// kind's code, with no runtime branch on the kind.
+enum TileKind : int32_t {
+  kTilesAll = 0,       // dense tangents, every query tile
+  kTilesNoisyCTZ = 1,  // clean-tangent-zero: tiles with a noisy row (q1 > L)
+  kTilesCleanCTZ = 2,  // clean-tangent-zero: tiles of clean rows only (primal only)
 };
 
 struct Sm100Params {
@@ -34,7 +45,7 @@ struct Sm100Params {
   float scale_log2e;     // scale * log2(e)
   uint64_t timeout_ns;   // bounded-wait limit
   int32_t fault_mode;    // test hook: 1 = skip the query-tile copies
-  int32_t clean_tangent_zero;  // tq, tk, tv vanish on rows < L (teacher-forcing layout)
+  int32_t tile_kind;     // TileKind: the query tiles this launch covers
   uint16_t qtile_order[kMaxQTiles];  // heaviest query tiles first
 };
 
