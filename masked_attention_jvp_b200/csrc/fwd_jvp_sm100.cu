@@ -35,6 +35,9 @@
 // [32g, 32g+32) is packed into S columns [32g, 32g+16) and P o tS into the same
 // columns of tS, so each thread only overwrites score columns it has read.
 //
+// Under clean-tangent-zero teacher forcing, the query tiles of clean rows need
+// no tangent at all; they run in a primal-only kernel further down.
+//
 // Every wait on an mbarrier is bounded by a time limit; on expiry the kernel
 // records an error code in a device word, drains its own in-flight copies and
 // MMAs, frees its tensor memory and returns.
@@ -191,12 +194,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, timeout_ns, site));
 }
 
-// KIND (a TileKind): dense tangents, or one of the two kinds of query tile of
-// clean-tangent-zero teacher forcing (the caller guarantees tq, tk, tv vanish on
-// rows < L). Each is its own instantiation: the dense kernel carries no trace of
-// the specialisation, and neither CTZ kernel branches on its tiles' kind at run
-// time (measured: the branching kernel took 16.0 ms on the TF frame-wise
-// workload, the two specialised launches 11.7 ms).
+// KIND (a TileKind): dense tangents (kTilesAll), or the query tiles with a noisy
+// row under clean-tangent-zero teacher forcing (kTilesNoisyCTZ: the caller
+// guarantees tq, tk, tv vanish on rows < L). Each is its own instantiation, so
+// the dense kernel carries no trace of the specialisation; the clean query
+// tiles have a kernel of their own (fwd_primal_sm100_kernel). Measured on the
+// TF frame-wise workload: one kernel branching on the kind of each tile took
+// 16.0 ms, the two specialised launches 12.0 ms.
 template <int D, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {
@@ -224,14 +228,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t t0, t1, t2, t3;
   const int32_t ntiles = qtile_key_tiles(p.geom, q0, q1, BN, t0, t1, t2, t3);
   const int32_t n0 = t1 - t0;
-  // Clean-tangent-zero teacher forcing: a tile of clean query rows has no
-  // tangent at all, and a key tile of clean tokens has tK = tV = 0.
+  // Clean-tangent-zero teacher forcing: a key tile of clean tokens has
+  // tK = tV = 0. (Tiles of clean query rows have no tangent at all and run in
+  // fwd_primal_sm100_kernel below.)
+  static_assert(KIND == kTilesAll || KIND == kTilesNoisyCTZ, "clean tiles run in the primal kernel");
   constexpr bool CTZ = KIND != kTilesAll;
-  constexpr bool no_tan = KIND == kTilesCleanCTZ;  // clean query rows: primal only
   auto clean_keys = [&](int32_t key0) { return CTZ && key0 + BN <= p.geom.L; };
   // The host partitions the query tiles by kind; a tile of the other kind is
   // refused before any barrier or TMEM use (the whole CTA leaves together).
-  if (CTZ && (q1 <= p.geom.L) != no_tan) {
+  if (CTZ && q1 <= p.geom.L) {
     if (threadIdx.x == 0) atomicCAS(&g_device_error, 0u, uint32_t(kErrTileKind));
     return;
   }
@@ -272,10 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sq = sbase + C::OFF_Q, stq = sbase + C::OFF_TQ;
     const bool load_q = p.fault_mode != 1;  // test hook: leave q_full unarmed
     if (load_q) {
-      mbar_arrive_expect_tx_if(leader, bar.q_full, no_tan ? C::Q_TX / 2 : C::Q_TX);
+      mbar_arrive_expect_tx_if(leader, bar.q_full, C::Q_TX);
       for (int c = 0; c < C::NB; ++c) {
         tma_load_3d(leader, sq + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
-        if (!no_tan) tma_load_3d(leader, stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
+        tma_load_3d(leader, stq + c * C::QBLK, &p.tm_tq, bar.q_full, c * 64, q0, bh);
       }
     }
     // Step j loads K|tK of key tile j (j < ntiles) into K stage j%2 and V|tV
@@ -351,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t i = j - 1;  // key tile whose value products this step issues
       bool have_p = i < 0;
       if (j < ntiles) {
-        const int s_mode = no_tan ? 2 : (clean_keys(tile_at(j, t0, n0, t2) * BN) ? 1 : 0);
+        const bool s_clean = clean_keys(tile_at(j, t0, n0, t2) * BN);
         const uint64_t dK = dK0 + uint64_t(((j & 1) * C::KT_STAGE) >> 4);
         const uint32_t dS = tS0 + (j & 1) * C::BUF_COLS;
 #pragma unroll
@@ -364,14 +369,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // 16 bf16 (32 bytes) per k-step inside a 128-byte swizzle atom, 64 per column block
           const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
           const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
-          if (s_mode == 0) {         // [S | Q tK^T] = Q [K;tK]^T, then tS += tQ K^T
+          if (!s_clean) {  // [S | Q tK^T] = Q [K;tK]^T, then tS += tQ K^T
             mma_ss(leader, dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
             mma_ss(leader, dS + BN, dTQ + qo, dK + ko, ID_TS, 1u);
-          } else if (s_mode == 1) {  // clean keys (tK = 0): S = Q K^T, tS = tQ K^T
+          } else {         // clean keys (tK = 0): S = Q K^T, tS = tQ K^T
             mma_ss(leader, dS, dQ + qo, dK + ko, ID_TS, kk > 0 ? 1u : 0u);
             mma_ss(leader, dS + BN, dTQ + qo, dK + ko, ID_TS, kk > 0 ? 1u : 0u);
-          } else {                   // no tangent in this query tile: S = Q K^T only
-            mma_ss(leader, dS, dQ + qo, dK + ko, ID_TS, kk > 0 ? 1u : 0u);
           }
         }
         if (!ok) break;
@@ -387,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dV = dV0 + uint64_t(((i & 1) * C::V_STAGE) >> 4);
         const uint32_t aP = tS0 + (i & 1) * C::BUF_COLS;
         const uint32_t first = i > 0 ? 1u : 0u;
-        const int v_mode = no_tan ? 2 : (clean_keys(tile_at(i, t0, n0, t2) * BN) ? 1 : 0);
+        const bool v_clean = clean_keys(tile_at(i, t0, n0, t2) * BN);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           if (kk == BN / 16 - kProbeLeadV && !have_x) {
@@ -398,14 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
           const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
-          if (v_mode == 0) {         // [O | T] += P [V | tV], then T += (P o tS) V
+          if (!v_clean) {  // [O | T] += P [V | tV], then T += (P o tS) V
             mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_OT, kk > 0 ? 1u : first);
             mma_ts(leader, tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, 1u);
-          } else if (v_mode == 1) {  // clean keys (tV = 0): O += P V, T += (P o tS) V
+          } else {         // clean keys (tV = 0): O += P V, T += (P o tS) V
             mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_T, kk > 0 ? 1u : first);
             mma_ts(leader, tmem + C::COL_T, aP + BN + pc, dV + vo, ID_T, kk > 0 ? 1u : first);
-          } else {                   // no tangent: O += P V only
-            mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_T, kk > 0 ? 1u : first);
           }
         }
         if (!ok) break;
@@ -453,13 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t cS = lane_addr + C::COL_S0 + b * C::BUF_COLS + 32 * g;
       const uint32_t cT = cS + BN;
       uint32_t rs[32], rt[32];
-      if (no_tan) {  // no score tangent was computed for this query tile
-        tmem_ld32(cS, rs);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rt[i] = 0u;
-      } else {
-        tmem_ld32x2(cS, cT, rs, rt);
-      }
+      tmem_ld32x2(cS, cT, rs, rt);
       float s[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(rs[i]);
@@ -526,30 +521,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this half's first 16 score columns.
       float ls[4] = {0.f, 0.f, 0.f, 0.f}, rsum[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[16], tk[16];
-      if (no_tan) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-          ls[i & 3] += pa + pb;
-          pk[i] = pack_bf16(pa, pb);
-        }
-        tmem_st16(cS, pk);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-          const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-          const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
-          const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
-          ls[i & 3] += pa + pb;
-          rsum[i & 3] += qa + qb;
-          pk[i] = pack_bf16(pa, pb);
-          tk[i] = pack_bf16(qa, qb);
-        }
-        tmem_st16(cS, pk);
-        tmem_st16(cT, tk);
+      for (int i = 0; i < 16; ++i) {
+        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+        const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
+        const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
+        ls[i & 3] += pa + pb;
+        rsum[i & 3] += qa + qb;
+        pk[i] = pack_bf16(pa, pb);
+        tk[i] = pack_bf16(qa, qb);
       }
+      tmem_st16(cS, pk);
+      tmem_st16(cT, tk);
       l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       r_run += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
       tmem_wait_st();
@@ -586,13 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
           uint32_t ro[32], rt[32];
-          if (no_tan) {  // T was never written: tO = 0
-            tmem_ld32(lane_addr + C::COL_O + c, ro);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) rt[i] = 0u;
-          } else {
-            tmem_ld32x2(lane_addr + C::COL_O + c, lane_addr + C::COL_T + c, ro, rt);
-          }
+          tmem_ld32x2(lane_addr + C::COL_O + c, lane_addr + C::COL_T + c, ro, rt);
           uint32_t po[16], pt[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -628,6 +606,377 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ================================================================ primal only
+// Query tiles of clean rows under clean-tangent-zero teacher forcing: their
+// tangents vanish, so tO = 0 and tLSE = 0 exactly, and only O = softmax(S) V
+// and LSE are computed. With no T accumulator and no score tangent, TMEM holds
+// O and four 64-column score buffers, and K and V have 4-deep rings of their
+// own: the MMA warp issues the scores of tile j, then O += P V of tile j - 3, so
+// the tensor core computes up to three tiles of scores ahead of the softmax.
+// Roles, softmax and masking are those of the JVP kernel above. Measured (ncu,
+// 4 heads of the TF frame-wise workload): tensor pipe 35% busy, exponential
+// unit 35%, issue slots 38% - the tile time is the latency of each warp's
+// serial per-tile chain (TMEM load, half-row max rendezvous, exponentials,
+// store, arrival), which the deeper score pipeline does not shorten; it ran
+// at the speed of the two-buffer JVP kernel's clean instantiation it replaces.
+// Two query tiles per CTA, each with a softmax warpgroup of its own (TMEM
+// holds both O tiles and their score buffers), would overlap those chains.
+constexpr int kPrimalBufs = 4;
+constexpr int kPrimalLag = kPrimalBufs - 1;
+
+template <int D>
+struct PCfg {
+  static constexpr int NS = kPrimalBufs;
+  static constexpr int NB = D / 64;
+  static constexpr int QBLK = BM * 128;
+  static constexpr int Q_BYTES = NB * QBLK;
+  static constexpr int KBLK = BN * 128;      // one column block of a K (or V) tile
+  static constexpr int K_STAGE = NB * KBLK;
+  static constexpr int V_STAGE = NB * KBLK;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * K_STAGE;
+  static constexpr int OFF_BAR = OFF_V + NS * V_STAGE;
+  // barriers: q_full, k_full[NS], v_full[NS], s_full[NS], p_full[NS], o_done[NS],
+  //           drain, pair[4 lane quarters][NS], pair_end[4 lane quarters]
+  static constexpr int NBAR = 1 + 5 * NS + 1 + 4 * NS + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_XCH = OFF_MISC + 16;  // [NS slots][2 halves][BM] fp32 row maxima
+  static constexpr int SMEM_BYTES = OFF_XCH + NS * 2 * BM * 4;
+  static constexpr uint32_t COL_O = 0;
+  static constexpr uint32_t COL_S0 = D;      // score buffer b: [COL_S0 + BN b, +BN)
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(COL_S0 + NS * BN <= TMEM_COLS, "tensor memory overflow");
+  static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+  static_assert(OFF_K % 1024 == 0 && K_STAGE % 1024 == 0, "128-byte swizzle needs 1 KiB aligned tiles");
+};
+
+struct PBarriers {
+  uint32_t q_full, k_full, v_full, s_full, p_full, o_done, drain, pair, pair_end;
+};
+
+template <int D>
+__device__ __forceinline__ PBarriers make_pbarriers(uint32_t base) {
+  constexpr int NS = PCfg<D>::NS;
+  PBarriers b;
+  b.q_full = base;
+  b.k_full = base + 8;
+  b.v_full = b.k_full + 8 * NS;
+  b.s_full = b.v_full + 8 * NS;
+  b.p_full = b.s_full + 8 * NS;
+  b.o_done = b.p_full + 8 * NS;
+  b.drain = b.o_done + 8 * NS;
+  b.pair = b.drain + 8;
+  b.pair_end = b.pair + 8 * 4 * NS;
+  return b;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_primal_sm100_kernel(const __grid_constant__ Sm100Params p) {
+  using C = PCfg<D>;
+  constexpr int NS = C::NS;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(&g_device_error, 0u, uint32_t(kErrSmemMisaligned));
+    return;
+  }
+  uint8_t *sgen = smem_raw;
+  const PBarriers bar = make_pbarriers<D>(sbase + C::OFF_BAR);
+  volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sgen + C::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + C::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int32_t bh = blockIdx.x / p.n_qtiles;
+  const int32_t qt = p.qtile_order[blockIdx.x % p.n_qtiles];
+  const int32_t q0 = qt * BM;
+  const int32_t q1 = min(q0 + BM, p.geom.N);
+  int32_t t0, t1, t2, t3;
+  const int32_t ntiles = qtile_key_tiles(p.geom, q0, q1, BN, t0, t1, t2, t3);
+  const int32_t n0 = t1 - t0;
+  // only clean query rows come here; the host partitions the tiles
+  if (p.tile_kind != kTilesCleanCTZ || q1 > p.geom.L) {
+    if (threadIdx.x == 0) atomicCAS(&g_device_error, 0u, uint32_t(kErrTileKind));
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar.q_full, 1);
+    for (int b = 0; b < NS; ++b) {
+      mbar_init(bar.k_full + 8 * b, 1);
+      mbar_init(bar.v_full + 8 * b, 1);
+      mbar_init(bar.s_full + 8 * b, 1);
+      mbar_init(bar.p_full + 8 * b, kSoftmaxWarps);
+      mbar_init(bar.o_done + 8 * b, 1);
+    }
+    mbar_init(bar.drain, 1);
+    for (int i = 0; i < 4 * NS; ++i) mbar_init(bar.pair + 8 * i, 2);
+    for (int i = 0; i < 4; ++i) mbar_init(bar.pair_end + 8 * i, 2);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint32_t leader = elect_one();
+    if (leader) {
+      prefetch_tmap(&p.tm_q);
+      prefetch_tmap(&p.tm_k);
+      prefetch_tmap(&p.tm_v);
+    }
+    const bool load_q = p.fault_mode != 1;  // test hook: leave q_full unarmed
+    if (load_q) {
+      mbar_arrive_expect_tx_if(leader, bar.q_full, C::Q_BYTES);
+      for (int c = 0; c < C::NB; ++c)
+        tma_load_3d(leader, sbase + C::OFF_Q + c * C::QBLK, &p.tm_q, bar.q_full, c * 64, q0, bh);
+    }
+    int32_t armed = 0;
+    for (int32_t j = 0; j < ntiles; ++j) {
+      const int b = j % NS;
+      const uint32_t ph = ((j / NS) - 1) & 1;  // phase of the previous use of stage b
+      const int32_t key0 = tile_at(j, t0, n0, t2) * BN;
+      // K stage b held tile j - NS: its scores must have completed
+      if (j >= NS && !warp_wait(bar.s_full + 8 * b, ph, abort_flag, p.timeout_ns, 12)) break;
+      mbar_arrive_expect_tx_if(leader, bar.k_full + 8 * b, C::K_STAGE);
+#pragma unroll
+      for (int c = 0; c < C::NB; ++c)
+        tma_load_3d(leader, sbase + C::OFF_K + b * C::K_STAGE + c * C::KBLK, &p.tm_k, bar.k_full + 8 * b,
+                    c * 64, key0, bh);
+      // V stage b held tile j - NS: its value product must have completed
+      if (j >= NS && !warp_wait(bar.o_done + 8 * b, ph, abort_flag, p.timeout_ns, 13)) {
+        armed = -(j + 1);  // K of tile j is in flight, V is not
+        break;
+      }
+      mbar_arrive_expect_tx_if(leader, bar.v_full + 8 * b, C::V_STAGE);
+#pragma unroll
+      for (int c = 0; c < C::NB; ++c)
+        tma_load_3d(leader, sbase + C::OFF_V + b * C::V_STAGE + c * C::KBLK, &p.tm_v, bar.v_full + 8 * b,
+                    c * 64, key0, bh);
+      armed = j + 1;
+    }
+    // Drain every copy this warp issued before the CTA releases its memory.
+    if (load_q) drain_wait(bar.q_full, 0, p.timeout_ns);
+    const int32_t k_armed = armed < 0 ? -armed : armed, v_armed = armed < 0 ? -armed - 1 : armed;
+    for (int32_t j = (k_armed > NS ? k_armed - NS : 0); j < k_armed; ++j)
+      drain_wait(bar.k_full + 8 * (j % NS), (j / NS) & 1, p.timeout_ns);
+    for (int32_t j = (v_armed > NS ? v_armed - NS : 0); j < v_armed; ++j)
+      drain_wait(bar.v_full + 8 * (j % NS), (j / NS) & 1, p.timeout_ns);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    const uint32_t leader = elect_one();
+    constexpr uint32_t ID_S = idesc_bf16_f32(BM, BN, 0);  // Q K^T
+    constexpr uint32_t ID_O = idesc_bf16_f32(BM, D, 1);   // P V, V read MN-major
+    const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+    const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::KBLK, 1024);
+    bool ok = warp_wait(bar.q_full, 0, abort_flag, p.timeout_ns, 14);
+    for (int32_t j = 0; ok && j < ntiles + kPrimalLag; ++j) {
+      if (j < ntiles) {
+        // Buffer j%NS last held P of tile j - NS, read by its value product,
+        // which was issued earlier (step j - 1): the tensor pipe runs in order.
+        const int b = j % NS;
+        if (!(ok = warp_wait(bar.k_full + 8 * b, (j / NS) & 1, abort_flag, p.timeout_ns, 15))) break;
+        tc_fence_after();
+        const uint64_t dK = dK0 + uint64_t((b * C::K_STAGE) >> 4);
+        const uint32_t dS = tmem + C::COL_S0 + b * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t qo = uint64_t(((kk >> 2) * C::QBLK + (kk & 3) * 32) >> 4);
+          const uint64_t ko = uint64_t(((kk >> 2) * C::KBLK + (kk & 3) * 32) >> 4);
+          mma_ss(leader, dS, dQ + qo, dK + ko, ID_S, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(leader, bar.s_full + 8 * b);
+      }
+      const int32_t i = j - kPrimalLag;
+      if (i >= 0) {
+        const int b = i % NS;
+        if (!(ok = warp_wait(bar.p_full + 8 * b, (i / NS) & 1, abort_flag, p.timeout_ns, 16))) break;
+        if (!(ok = warp_wait(bar.v_full + 8 * b, (i / NS) & 1, abort_flag, p.timeout_ns, 17))) break;
+        tc_fence_after();
+        const uint64_t dV = dV0 + uint64_t((b * C::V_STAGE) >> 4);
+        const uint32_t aP = tmem + C::COL_S0 + b * BN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
+          const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
+          mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_O, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(leader, bar.o_done + 8 * b);
+      }
+    }
+    tc_commit(leader, bar.drain);
+    drain_wait(bar.drain, 0, p.timeout_ns);
+  } else {
+    // ------------------------------------------------- softmax + epilogue
+    const int g = (warp - 2) >> 2;
+    const int sub = warp & 3;
+    const int row = sub * 32 + lane;
+    const int32_t q = q0 + row;
+    const uint32_t lane_addr = tmem + (uint32_t(sub * 32) << 16);
+    float *xch = reinterpret_cast<float *>(sgen + C::OFF_XCH);  // [slot][half][row]
+    int32_t a0, b0, a1, b1;
+    if (q < p.geom.N) {
+      row_key_ranges(p.geom, q, a0, b0, a1, b1);
+    } else {
+      a0 = 0;
+      b0 = p.geom.N;
+      a1 = b1 = 0;
+    }
+    const float sl2 = p.scale_log2e;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+    for (int32_t j = 0; j < ntiles; ++j) {
+      const int b = j % NS;
+      if (!warp_wait(bar.s_full + 8 * b, (j / NS) & 1, abort_flag, p.timeout_ns, 18)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int32_t kh = tile_at(j, t0, n0, t2) * BN + 32 * g;
+      const uint32_t cS = lane_addr + C::COL_S0 + b * BN + 32 * g;
+      uint32_t rs[32];
+      tmem_ld32(cS, rs);
+      float s[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(rs[i]);
+      const uint32_t vis = range_bits(a0 - kh, b0 - kh) | range_bits(a1 - kh, b1 - kh);
+      if (vis != 0xffffffffu) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] = ((vis >> i) & 1u) ? s[i] : -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
+      const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      xch[(b * 2 + g) * BM + row] = hmax;
+      if (!pair_sync(bar.pair + 8 * (sub * NS + b), (j / NS) & 1, lane, abort_flag, p.timeout_ns, 19)) {
+        ok = false;
+        break;
+      }
+      const float tmax = fmaxf(hmax, xch[(b * 2 + (g ^ 1)) * BM + row]);
+      const float m_tile = tmax * sl2;
+      const bool grow = m_tile > m_run + kRescaleThreshold;
+      const bool had_acc = m_run != -INFINITY;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = had_acc ? ex2(m_run - m_tile) : 0.f;
+        l_run *= alpha;
+        m_run = m_tile;
+      }
+      if (__any_sync(0xffffffffu, grow && had_acc) && j > 0) {
+        // O must be scaled by alpha once every earlier value product has landed:
+        // those run in order, so the one of tile j - 1 is enough. Each
+        // warpgroup scales its half of the columns.
+        const int pb = (j - 1) % NS;
+        if (!warp_wait(bar.o_done + 8 * pb, ((j - 1) / NS) & 1, abort_flag, p.timeout_ns, 20)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + C::COL_O + c, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(lane_addr + C::COL_O + c, r);
+        }
+      }
+      const float ref = (m_run == -INFINITY) ? 0.f : m_run;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
+        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
+        ls[i & 3] += pa + pb;
+        pk[i] = pack_bf16(pa, pb);
+      }
+      tmem_st16(cS, pk);
+      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.p_full + 8 * b);
+    }
+
+    if (ok && ntiles > 0) {
+      // Combine the two halves' sums. Slot ntiles%NS... is free: its last
+      // reader (tile ntiles - NS) passed its rendezvous long before.
+      const int sl = ntiles % NS;
+      xch[(sl * 2 + g) * BM + row] = l_run;
+      bool got = pair_sync(bar.pair_end + 8 * sub, 0, lane, abort_flag, p.timeout_ns, 21);
+      const float l_tot = l_run + xch[(sl * 2 + (g ^ 1)) * BM + row];
+      const int32_t last = ntiles - 1;
+      if (got)
+        got = wait_bounded(bar.o_done + 8 * (last % NS), (last / NS) & 1, abort_flag, p.timeout_ns, 22);
+      if (__all_sync(0xffffffffu, got)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_tot;
+        const bool store = q < p.geom.N;
+        const size_t rowoff = (size_t(bh) * p.geom.N + (store ? q : 0)) * D;
+        uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
+        uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
+#pragma unroll 1
+        for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
+          uint32_t ro[32];
+          tmem_ld32(lane_addr + C::COL_O + c, ro);
+          uint32_t po[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            po[i] = pack_bf16(__uint_as_float(ro[2 * i]) * inv_l, __uint_as_float(ro[2 * i + 1]) * inv_l);
+          if (store) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              orow[c / 8 + v] = make_uint4(po[4 * v], po[4 * v + 1], po[4 * v + 2], po[4 * v + 3]);
+              torow[c / 8 + v] = make_uint4(0u, 0u, 0u, 0u);  // clean rows: the tangent vanishes
+            }
+          }
+        }
+        if (store && g == 0) {
+          const size_t ri = size_t(bh) * p.geom.N + q;
+          p.lse[ri] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+          p.tlse[ri] = 0.f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_primal_impl(const Sm100Params &p, cudaStream_t stream) {
+  using C = PCfg<D>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_primal_sm100_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
+  fwd_primal_sm100_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int D, int KIND>
 cudaError_t launch_impl(const Sm100Params &p, cudaStream_t stream) {
   using C = Cfg<D>;
@@ -649,10 +998,10 @@ cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t strea
   switch (p.tile_kind * 256 + D) {
     case kTilesAll * 256 + 128: return launch_impl<128, kTilesAll>(p, stream);
     case kTilesNoisyCTZ * 256 + 128: return launch_impl<128, kTilesNoisyCTZ>(p, stream);
-    case kTilesCleanCTZ * 256 + 128: return launch_impl<128, kTilesCleanCTZ>(p, stream);
+    case kTilesCleanCTZ * 256 + 128: return launch_primal_impl<128>(p, stream);
     case kTilesAll * 256 + 64: return launch_impl<64, kTilesAll>(p, stream);
     case kTilesNoisyCTZ * 256 + 64: return launch_impl<64, kTilesNoisyCTZ>(p, stream);
-    case kTilesCleanCTZ * 256 + 64: return launch_impl<64, kTilesCleanCTZ>(p, stream);
+    case kTilesCleanCTZ * 256 + 64: return launch_primal_impl<64>(p, stream);
     default: return cudaErrorInvalidValue;
   }
 }
