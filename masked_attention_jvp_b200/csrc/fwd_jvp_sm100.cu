@@ -609,18 +609,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ================================================================ primal only
 // Query tiles of clean rows under clean-tangent-zero teacher forcing: their
 // tangents vanish, so tO = 0 and tLSE = 0 exactly, and only O = softmax(S) V
-// and LSE are computed. With no T accumulator and no score tangent, TMEM holds
-// O and four 64-column score buffers, and K and V have 4-deep rings of their
-// own: the MMA warp issues the scores of tile j, then O += P V of tile j - 3, so
-// the tensor core computes up to three tiles of scores ahead of the softmax.
-// Roles, softmax and masking are those of the JVP kernel above. Measured (ncu,
-// 4 heads of the TF frame-wise workload): tensor pipe 35% busy, exponential
-// unit 35%, issue slots 38% - the tile time is the latency of each warp's
-// serial per-tile chain (TMEM load, half-row max rendezvous, exponentials,
-// store, arrival), which the deeper score pipeline does not shorten; it ran
-// at the speed of the two-buffer JVP kernel's clean instantiation it replaces.
-// Two query tiles per CTA, each with a softmax warpgroup of its own (TMEM
-// holds both O tiles and their score buffers), would overlap those chains.
+// and LSE are computed.
+// The two softmax warpgroups split the key tiles, not the keys of a tile:
+// warpgroup g takes tiles j = g (mod 2), each thread a whole 64-key row of
+// them, with its own running max m_g, sum l_g and accumulator O_g in TMEM.
+// The two online softmaxes run side by side with no rendezvous per tile; the
+// epilogue merges them once: with m = max(m_0, m_1) and a_g = 2^(m_g - m),
+//   O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1),  LSE = ln 2 (m + log2 of that sum).
+// (Measured against the JVP kernel's scheme, where the two warpgroups take the
+// two 32-key halves of every tile and meet each tile to agree on a row max: the
+// per-tile chain of a warp - TMEM load, rendezvous, exponentials, store - was
+// the limit, with the tensor pipe 35% busy.)
+// TMEM: O_0 [0, D) | O_1 [D, 2D) | four 64-column score buffers. K and V have
+// 4-deep rings; the MMA warp issues the scores of tile j, then O_(i%2) += P V
+// of tile i = j - 3, so the tensor core runs up to three tiles of scores ahead.
+// Roles and masking are those of the JVP kernel above.
 constexpr int kPrimalBufs = 4;
 constexpr int kPrimalLag = kPrimalBufs - 1;
 
@@ -638,21 +641,22 @@ struct PCfg {
   static constexpr int OFF_V = OFF_K + NS * K_STAGE;
   static constexpr int OFF_BAR = OFF_V + NS * V_STAGE;
   // barriers: q_full, k_full[NS], v_full[NS], s_full[NS], p_full[NS], o_done[NS],
-  //           drain, pair[4 lane quarters][NS], pair_end[4 lane quarters]
-  static constexpr int NBAR = 1 + 5 * NS + 1 + 4 * NS + 4;
+  //           drain, pair_end[4 lane quarters]
+  static constexpr int NBAR = 1 + 5 * NS + 1 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_XCH = OFF_MISC + 16;  // [NS slots][2 halves][BM] fp32 row maxima
-  static constexpr int SMEM_BYTES = OFF_XCH + NS * 2 * BM * 4;
-  static constexpr uint32_t COL_O = 0;
-  static constexpr uint32_t COL_S0 = D;      // score buffer b: [COL_S0 + BN b, +BN)
+  static constexpr int OFF_XCH = OFF_MISC + 16;  // [m, l][2 warpgroups][BM] fp32
+  static constexpr int SMEM_BYTES = OFF_XCH + 2 * 2 * BM * 4;
+  static constexpr uint32_t COL_O = 0;       // O_g at COL_O + g D
+  static constexpr uint32_t COL_S0 = 2 * D;  // score buffer b: [COL_S0 + BN b, +BN)
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(COL_S0 + NS * BN <= TMEM_COLS, "tensor memory overflow");
   static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
   static_assert(OFF_K % 1024 == 0 && K_STAGE % 1024 == 0, "128-byte swizzle needs 1 KiB aligned tiles");
+  static_assert(NS % 2 == 0, "buffer b serves warpgroup b % 2");
 };
 
 struct PBarriers {
-  uint32_t q_full, k_full, v_full, s_full, p_full, o_done, drain, pair, pair_end;
+  uint32_t q_full, k_full, v_full, s_full, p_full, o_done, drain, pair_end;
 };
 
 template <int D>
@@ -666,8 +670,7 @@ __device__ __forceinline__ PBarriers make_pbarriers(uint32_t base) {
   b.p_full = b.s_full + 8 * NS;
   b.o_done = b.p_full + 8 * NS;
   b.drain = b.o_done + 8 * NS;
-  b.pair = b.drain + 8;
-  b.pair_end = b.pair + 8 * 4 * NS;
+  b.pair_end = b.drain + 8;
   return b;
 }
 
@@ -707,11 +710,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar.k_full + 8 * b, 1);
       mbar_init(bar.v_full + 8 * b, 1);
       mbar_init(bar.s_full + 8 * b, 1);
-      mbar_init(bar.p_full + 8 * b, kSoftmaxWarps);
+      mbar_init(bar.p_full + 8 * b, kSoftmaxWarps / 2);  // the four warps of one warpgroup
       mbar_init(bar.o_done + 8 * b, 1);
     }
     mbar_init(bar.drain, 1);
-    for (int i = 0; i < 4 * NS; ++i) mbar_init(bar.pair + 8 * i, 2);
     for (int i = 0; i < 4; ++i) mbar_init(bar.pair_end + 8 * i, 2);
     *abort_flag = 0;
     fence_mbar_init();
@@ -804,11 +806,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t dV = dV0 + uint64_t((b * C::V_STAGE) >> 4);
         const uint32_t aP = tmem + C::COL_S0 + b * BN;
+        const uint32_t dO = tmem + C::COL_O + (i & 1) * D;  // warpgroup i%2's accumulator
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t vo = uint64_t((kk * 16 * 128) >> 4);  // 16 keys of 128-byte rows
           const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;   // packed P columns of keys 16kk..
-          mma_ts(leader, tmem + C::COL_O, aP + pc, dV + vo, ID_O, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(leader, dO, aP + pc, dV + vo, ID_O, (i > 1 || kk > 0) ? 1u : 0u);
         }
         tc_commit(leader, bar.o_done + 8 * b);
       }
@@ -817,12 +820,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     drain_wait(bar.drain, 0, p.timeout_ns);
   } else {
     // ------------------------------------------------- softmax + epilogue
-    const int g = (warp - 2) >> 2;
+    const int g = (warp - 2) >> 2;  // this warpgroup takes key tiles j = g (mod 2)
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
     const int32_t q = q0 + row;
     const uint32_t lane_addr = tmem + (uint32_t(sub * 32) << 16);
-    float *xch = reinterpret_cast<float *>(sgen + C::OFF_XCH);  // [slot][half][row]
+    const uint32_t cO = lane_addr + C::COL_O + g * D;
+    float *xch = reinterpret_cast<float *>(sgen + C::OFF_XCH);  // [m, l][warpgroup][row]
     int32_t a0, b0, a1, b1;
     if (q < p.geom.N) {
       row_key_ranges(p.geom, q, a0, b0, a1, b1);
@@ -832,41 +836,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       a1 = b1 = 0;
     }
     const float sl2 = p.scale_log2e;
-    float m_run = -INFINITY;
+    float m_run = -INFINITY;  // of this warpgroup's tiles, possibly stale by < 2^8
     float l_run = 0.f;
     bool ok = true;
-    for (int32_t j = 0; j < ntiles; ++j) {
+    for (int32_t j = g; j < ntiles; j += 2) {
       const int b = j % NS;
       if (!warp_wait(bar.s_full + 8 * b, (j / NS) & 1, abort_flag, p.timeout_ns, 18)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int32_t kh = tile_at(j, t0, n0, t2) * BN + 32 * g;
-      const uint32_t cS = lane_addr + C::COL_S0 + b * BN + 32 * g;
-      uint32_t rs[32];
-      tmem_ld32(cS, rs);
-      float s[32];
+      const int32_t kh = tile_at(j, t0, n0, t2) * BN;
+      const uint32_t cS = lane_addr + C::COL_S0 + b * BN;
+      uint32_t ra[32], rb[32];
+      tmem_ld32x2(cS, cS + 32, ra, rb);
+      float s[64];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(rs[i]);
-      const uint32_t vis = range_bits(a0 - kh, b0 - kh) | range_bits(a1 - kh, b1 - kh);
-      if (vis != 0xffffffffu) {
+      for (int i = 0; i < 32; ++i) {
+        s[i] = __uint_as_float(ra[i]);
+        s[32 + i] = __uint_as_float(rb[i]);
+      }
+      // keys of this tile the row may see; mask only where some are hidden
+      const uint32_t v0 = range_bits(a0 - kh, b0 - kh) | range_bits(a1 - kh, b1 - kh);
+      const uint32_t v1 = range_bits(a0 - kh - 32, b0 - kh - 32) | range_bits(a1 - kh - 32, b1 - kh - 32);
+      if ((v0 & v1) != 0xffffffffu) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = ((vis >> i) & 1u) ? s[i] : -INFINITY;
+        for (int i = 0; i < 32; ++i) {
+          s[i] = ((v0 >> i) & 1u) ? s[i] : -INFINITY;
+          s[32 + i] = ((v1 >> i) & 1u) ? s[32 + i] : -INFINITY;
+        }
       }
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
+      for (int i = 0; i < 8; ++i)
+        mx[i] = fmaxf(fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24])),
+                      fmaxf(fmaxf(s[i + 32], s[i + 40]), fmaxf(s[i + 48], s[i + 56])));
 #pragma unroll
       for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
-      const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      xch[(b * 2 + g) * BM + row] = hmax;
-      if (!pair_sync(bar.pair + 8 * (sub * NS + b), (j / NS) & 1, lane, abort_flag, p.timeout_ns, 19)) {
-        ok = false;
-        break;
-      }
-      const float tmax = fmaxf(hmax, xch[(b * 2 + (g ^ 1)) * BM + row]);
-      const float m_tile = tmax * sl2;
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       const bool grow = m_tile > m_run + kRescaleThreshold;
       const bool had_acc = m_run != -INFINITY;
       float alpha = 1.f;
@@ -875,36 +882,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run *= alpha;
         m_run = m_tile;
       }
-      if (__any_sync(0xffffffffu, grow && had_acc) && j > 0) {
-        // O must be scaled by alpha once every earlier value product has landed:
-        // those run in order, so the one of tile j - 1 is enough. Each
-        // warpgroup scales its half of the columns.
-        const int pb = (j - 1) % NS;
-        if (!warp_wait(bar.o_done + 8 * pb, ((j - 1) / NS) & 1, abort_flag, p.timeout_ns, 20)) {
+      if (__any_sync(0xffffffffu, grow && had_acc) && j >= 2) {
+        // O_g must be scaled once this warpgroup's previous tile (j - 2) has
+        // landed in it (value products complete in order).
+        const int pb = (j - 2) % NS;
+        if (!warp_wait(bar.o_done + 8 * pb, ((j - 2) / NS) & 1, abort_flag, p.timeout_ns, 20)) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
+        for (int c = 0; c < D; c += 32) {
           uint32_t r[32];
-          tmem_ld32(lane_addr + C::COL_O + c, r);
+          tmem_ld32(cO + c, r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(lane_addr + C::COL_O + c, r);
+          tmem_st32(cO + c, r);
         }
       }
       const float ref = (m_run == -INFINITY) ? 0.f : m_run;
+      // P = 2^(s*scale*log2e - ref) in bf16: keys 0-31 packed into columns
+      // 0-15, keys 32-63 into columns 32-47 (the layout the value MMA reads)
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[16];
+      uint32_t pk0[16], pk1[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
         const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-        ls[i & 3] += pa + pb;
-        pk[i] = pack_bf16(pa, pb);
+        const float pc = ex2(fmaf(s[32 + 2 * i], sl2, -ref));
+        const float pd = ex2(fmaf(s[32 + 2 * i + 1], sl2, -ref));
+        ls[i & 3] += (pa + pb) + (pc + pd);
+        pk0[i] = pack_bf16(pa, pb);
+        pk1[i] = pack_bf16(pc, pd);
       }
-      tmem_st16(cS, pk);
+      tmem_st16(cS, pk0);
+      tmem_st16(cS + 32, pk1);
       l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();
@@ -913,30 +925,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (ok && ntiles > 0) {
-      // Combine the two halves' sums. Slot ntiles%NS... is free: its last
-      // reader (tile ntiles - NS) passed its rendezvous long before.
-      const int sl = ntiles % NS;
-      xch[(sl * 2 + g) * BM + row] = l_run;
+      // Merge the two warpgroups' partial softmaxes (a warpgroup without tiles,
+      // or whose tiles the row cannot see, has m = -inf and contributes 0).
+      xch[(0 * 2 + g) * BM + row] = m_run;
+      xch[(1 * 2 + g) * BM + row] = l_run;
       bool got = pair_sync(bar.pair_end + 8 * sub, 0, lane, abort_flag, p.timeout_ns, 21);
-      const float l_tot = l_run + xch[(sl * 2 + (g ^ 1)) * BM + row];
+      const float m_o = xch[(0 * 2 + (g ^ 1)) * BM + row], l_o = xch[(1 * 2 + (g ^ 1)) * BM + row];
+      const float m_0 = g ? m_o : m_run, m_1 = g ? m_run : m_o;
+      const float l_0 = g ? l_o : l_run, l_1 = g ? l_run : l_o;
+      const float m = fmaxf(m_0, m_1);
+      const bool has0 = m_0 != -INFINITY, has1 = m_1 != -INFINITY;
+      const float f0 = has0 ? ex2(m_0 - m) : 0.f, f1 = has1 ? ex2(m_1 - m) : 0.f;
+      const float l_tot = f0 * l_0 + f1 * l_1;
       const int32_t last = ntiles - 1;
       if (got)
         got = wait_bounded(bar.o_done + 8 * (last % NS), (last / NS) & 1, abort_flag, p.timeout_ns, 22);
       if (__all_sync(0xffffffffu, got)) {
         tc_fence_after();
-        const float inv_l = 1.f / l_tot;
+        const float w0 = f0 / l_tot, w1 = f1 / l_tot;
         const bool store = q < p.geom.N;
         const size_t rowoff = (size_t(bh) * p.geom.N + (store ? q : 0)) * D;
         uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
         uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
+        // warpgroup g writes output columns [g D/2, (g+1) D/2)
 #pragma unroll 1
         for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
-          uint32_t ro[32];
-          tmem_ld32(lane_addr + C::COL_O + c, ro);
+          uint32_t r0[32], r1[32];
+          tmem_ld32x2(lane_addr + C::COL_O + c, lane_addr + C::COL_O + D + c, r0, r1);
           uint32_t po[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            po[i] = pack_bf16(__uint_as_float(ro[2 * i]) * inv_l, __uint_as_float(ro[2 * i + 1]) * inv_l);
+          for (int i = 0; i < 16; ++i) {
+            // select, not multiply: an accumulator never written holds garbage
+            const float x0 = has0 ? __uint_as_float(r0[2 * i]) * w0 : 0.f;
+            const float y0 = has0 ? __uint_as_float(r0[2 * i + 1]) * w0 : 0.f;
+            const float x1 = has1 ? __uint_as_float(r1[2 * i]) * w1 : 0.f;
+            const float y1 = has1 ? __uint_as_float(r1[2 * i + 1]) * w1 : 0.f;
+            po[i] = pack_bf16(x0 + x1, y0 + y1);
+          }
           if (store) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -947,7 +972,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (store && g == 0) {
           const size_t ri = size_t(bh) * p.geom.N + q;
-          p.lse[ri] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+          p.lse[ri] = (m + __log2f(l_tot)) * 0.69314718055994530942f;
           p.tlse[ri] = 0.f;
         }
       }
