@@ -146,6 +146,19 @@ def time_oracle(w, target_s=15.0, host_inputs=None):
     return fl / dt / 1e12, dt, rows.numel(), threads, desc
 
 
+def host_cpu() -> dict:
+    """The host CPU's model name and logical core count (for the oracle baseline)."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
     """SM clock and clock-event reasons of this process's GPU, sampled every
@@ -415,6 +428,7 @@ def bench_gpu(args, rank, world, local_rank):
         return None
     peaks, src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     kernel_ms = statistics.mean(per)
     achieved = fl / (kernel_ms / 1e3) / 1e12
     clocks = clk.summary()
@@ -432,6 +446,8 @@ def bench_gpu(args, rank, world, local_rank):
         "gpu_launches": args.steps,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4),
+                     "frac_of_sustained": round(achieved / peak_sustained, 4),
+                     "peak_sustained": peak_sustained,
                      "traffic": MEASURED_TRAFFIC.get((w.name, kernel_sources_hash())),
                      "kernel_sources_sha256": kernel_sources_hash(),
                      "peak_source": f"{src} bf16 burst (cuBLAS)", "kernel": "fwd_jvp_sm100_kernel<128>"},
@@ -452,11 +468,15 @@ def bench_gpu(args, rank, world, local_rank):
         line["products_tflop_per_step"] = round(ctz_product_flops(w) / 1e12, 3)
         line["roofline"]["achieved"] = round(ctz_product_flops(w) / (kernel_ms / 1e3) / 1e12, 2)
         line["roofline"]["frac"] = round(line["roofline"]["achieved"] / peak, 4)
+        line["roofline"]["frac_of_sustained"] = round(line["roofline"]["achieved"] / peak_sustained, 4)
         line["roofline"]["note"] = "achieved counts only the products the kernel must do"
     if world == 1 and not args.no_cpu_baseline:
         tf, dt, nrows, threads, desc = time_oracle(w, host_inputs=host)
         line["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": threads,
-                                "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+                                "kind": "oracle", "sample": desc, "seconds": round(dt, 2),
+                                "rows_per_s": round(nrows / dt, 1),
+                                "extrapolated_full_call_s": round(fl / (tf * 1e12), 1),
+                                "host": host_cpu()}
     return line
 
 
@@ -488,7 +508,7 @@ def bench_reference(args, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": workload_config(w),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "host": host_cpu()},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

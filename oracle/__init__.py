@@ -180,3 +180,26 @@ def attn_bwd(q, k, v, dout, mask, scale=None):
     if rc != 0:
         raise ValueError("oracle: rejected arguments")
     return dq, dk, dv, delta
+
+
+def out_proj_jvp(x, tx, w, bias=None):
+    """Output projection of the attention block in primal-tangent form.
+
+    Causal-rCM, section 3.2.2 ("JVP FSDP2"): the JVP runs layer by layer, each
+    layer taking and returning a (primal, tangent) pair. The projection after
+    attention is linear, so its tangent is the same map without the bias:
+        y = x W^T + b,   ty = tx W^T.
+    x, tx: [M, K] (tokens x H*D, the attention output in token-major layout);
+    w: [C, K] (the layer's weight); bias: [C] or None. Returns (y, ty) as fp64
+    numpy arrays [M, C]; the matmul is numpy's, in fp64, on the exact input
+    values."""
+    def f64(t):  # exact widening of bf16 / fp32 values
+        if isinstance(t, torch.Tensor):
+            return t.detach().cpu().to(torch.float64).numpy()
+        return np.asarray(t, np.float64)
+
+    x64, tx64, w64 = f64(x), f64(tx), f64(w)
+    y = x64 @ w64.T
+    if bias is not None:
+        y = y + f64(bias)[None, :]
+    return y, tx64 @ w64.T
