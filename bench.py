@@ -348,6 +348,37 @@ def bench_backward(w, ins, o, lse, steps, peaks):
             "executed_products_tflop": round(14 * w.D * pairs / 1e12, 3)}
 
 
+# ------------------------------------------------------------ output projection
+def bench_out_proj(w, dev, steps, peaks):
+    """Output projection in primal-tangent form on the workload's tokens:
+    y = x W^T + b, ty = tx W^T with x, tx [B*N, H*D] and W [H*D, H*D] (the
+    model width; Wan-1.3B: 1536). Two GEMMs of 2*M*K*C flops each."""
+    import masked_attention_jvp_b200 as caj
+    M, K = w.B * w.N, w.H * w.D
+    C = K
+    g = torch.Generator(device=dev).manual_seed(w.seed + 3)
+    x, tx = (torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16) for _ in range(2))
+    wt = (torch.randn(C, K, device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
+    b = torch.randn(C, device=dev, generator=g).to(torch.bfloat16)
+    out = (torch.empty(M, C, device=dev, dtype=torch.bfloat16), torch.empty(M, C, device=dev, dtype=torch.bfloat16))
+    for _ in range(3):
+        caj.out_proj_jvp(x, tx, wt, b, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        caj.out_proj_jvp(x, tx, wt, b, out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    fl = 2 * 2 * M * K * C
+    tf = fl / (ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    return {"op": "y = x W^T + b, ty = tx W^T (cuBLASLt, bias epilogue)", "M": M, "K": K, "C": C,
+            "ms": round(ms, 4), "bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(tf / peak, 4)}
+
+
 # ------------------------------------------------------------------ GPU arm
 def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
     """Same metric through the public API from pinned host buffers: every step
@@ -458,6 +489,8 @@ def bench_gpu(args, rank, world, local_rank):
     if not args.no_prologue:
         line["prologue"] = bench_prologue(w, dev, args.steps, peaks)
         line["gpu_launches_prologue"] = args.steps
+    if not args.no_out_proj and not args.clean_tangent_zero:
+        line["out_proj"] = bench_out_proj(w, dev, args.steps, peaks)
     if args.clean_tangent_zero:
         # one launch for the query tiles with a noisy row, one for the clean ones
         L = w.mask.n_frames * w.mask.tokens_per_frame
@@ -532,6 +565,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-prologue", action="store_true", help="skip the prologue kernel's measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward kernels' measurement")
+    ap.add_argument("--no-out-proj", action="store_true", help="skip the output projection's measurement")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (small cases for ncu section captures)")
     ap.add_argument("--clean-tangent-zero", action="store_true",

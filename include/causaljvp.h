@@ -84,12 +84,19 @@ typedef struct {
  * clean tokens skip Q tK^T and P tV. With the guarantee the results equal the
  * dense definition; without it they do not.
  */
-typedef enum { CAJ_FLAG_CLEAN_TANGENT_ZERO = 1 } caj_flags;
+/*
+ * CAJ_FLAG_TOKEN_MAJOR_OUT: o and to are written token-major, [B, N, H, D]
+ * (= [B, N, H*D], the input layout of the output projection,
+ * caj_out_proj_jvp) instead of [B, H, N, D]. lse and tlse keep [B, H, N].
+ * Not accepted by caj_attn_fwd_jvp_host.
+ */
+typedef enum { CAJ_FLAG_CLEAN_TANGENT_ZERO = 1, CAJ_FLAG_TOKEN_MAJOR_OUT = 2 } caj_flags;
 
 /*
  * Forward + JVP of block-causal attention (appendix B eq. 42-45, Algorithm 1).
  *   in : q, k, v, tq, tk, tv   [B,H,N,D] of prob->dtype, read only
  *   out: o, to                 [B,H,N,D] of prob->dtype, fully overwritten
+ *                              ([B,N,H,D] with CAJ_FLAG_TOKEN_MAJOR_OUT)
  *        lse, tlse             [B,H,N] fp32, fully overwritten
  * Supported: D in {64, 128}; dtype BF16 (tensor-core path, fp32 accumulation)
  * or F32 (CUDA-core fp32 path); N == n_frames*tokens_per_frame*(tf_layout?2:1);
@@ -133,6 +140,31 @@ caj_status caj_attn_fwd_jvp_host(const void *q, const void *k, const void *v,
                                  const caj_problem *prob, const caj_mask_desc *mask,
                                  void *o, void *to, float *lse, float *tlse,
                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Output projection of the attention block in primal-tangent form. Causal-rCM
+ * runs the JVP layer by layer, each layer mapping a (primal, tangent) pair to a
+ * pair (section 3.2.2, "JVP FSDP2"); the projection after attention is
+ * linear, so its tangent is the same map without the bias:
+ *   y = x W^T + b,   ty = tx W^T
+ *   in : x, tx   [M, K] bf16 row-major: M = B*N tokens, K = H*D (the attention
+ *                output written with CAJ_FLAG_TOKEN_MAJOR_OUT)
+ *        w       [C, K] bf16 row-major (the layer's weight)
+ *        bias    [C] bf16, or null for none
+ *   out: y, ty   [M, C] bf16, fully overwritten
+ * Two bf16 GEMMs with fp32 accumulation (cuBLASLt, bias fused as its
+ * epilogue). No workspace: nothing is allocated per call. Pointers 16-byte
+ * aligned; K and C multiples of 8 (CAJ_ERR_UNSUPPORTED otherwise). Returns
+ * CAJ_OK once enqueued on `stream`, CAJ_ERR_INVALID_ARG without launching,
+ * or CAJ_ERR_CUDA (cuBLASLt refused; caj_last_cuda_error names its status).
+ */
+typedef struct {
+  int64_t M;
+  int32_t K, C;
+} caj_linear_shape;
+
+caj_status caj_out_proj_jvp(const void *x, const void *tx, const void *w, const void *bias,
+                            const caj_linear_shape *shape, void *y, void *ty, void *stream);
 
 /*
  * Attention-block prologue in primal-tangent form. Causal-rCM implements the

@@ -28,7 +28,7 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_bwd", "qk_norm_rope_jvp", "MaskDesc", "CajError", "visible_pairs",
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -74,19 +74,24 @@ def device_status(stream: Optional[torch.cuda.Stream] = None):
     _lib.check(_lib.lib().caj_last_device_status(ctypes.c_void_p(s)), "caj_last_device_status")
 
 
-def _problem(q: torch.Tensor, scale: Optional[float], clean_tangent_zero: bool = False) -> _lib.ProblemC:
+def _problem(q: torch.Tensor, scale: Optional[float], clean_tangent_zero: bool = False,
+             token_major_out: bool = False) -> _lib.ProblemC:
     B, H, N, D = q.shape
-    flags = _lib.CAJ_FLAG_CLEAN_TANGENT_ZERO if clean_tangent_zero else 0
+    flags = (_lib.CAJ_FLAG_CLEAN_TANGENT_ZERO if clean_tangent_zero else 0) | \
+        (_lib.CAJ_FLAG_TOKEN_MAJOR_OUT if token_major_out else 0)
     return _lib.ProblemC(B, H, N, D, _DTYPES[q.dtype], float(scale) if scale else 0.0, flags)
 
 
 def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optional[float] = None,
-                     stream: Optional[torch.cuda.Stream] = None, clean_tangent_zero: bool = False) -> None:
+                     stream: Optional[torch.cuda.Stream] = None, clean_tangent_zero: bool = False,
+                     token_major_out: bool = False) -> None:
     """Writes into caller-provided CUDA tensors o, to [B,H,N,D] and lse, tlse [B,H,N] fp32.
 
     clean_tangent_zero: teacher-forcing layout only; the caller guarantees that
     tq, tk, tv are zero on the clean half, and the kernel skips the products
-    that vanish (clean query tiles compute only the primal)."""
+    that vanish (clean query tiles compute only the primal).
+    token_major_out: o and to are [B,N,H,D] (the output projection's input
+    layout, see out_proj_jvp) instead of [B,H,N,D]."""
     ins = (q, k, v, tq, tk, tv)
     for t in ins + (o, to, lse, tlse):
         if not t.is_cuda:
@@ -95,13 +100,15 @@ def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optiona
             raise ValueError("attn_fwd_jvp_out: tensors must be contiguous")
     if q.dtype not in _DTYPES or any(t.dtype != q.dtype for t in ins + (o, to)):
         raise ValueError("attn_fwd_jvp_out: q..tv, o, to must share one dtype (bf16 or fp32)")
-    if any(t.shape != q.shape for t in ins + (o, to)):
+    B, H, N, D = q.shape
+    out_shape = (B, N, H, D) if token_major_out else (B, H, N, D)
+    if any(t.shape != q.shape for t in ins) or o.shape != out_shape or to.shape != out_shape:
         raise ValueError("attn_fwd_jvp_out: shape mismatch")
     if lse.dtype != torch.float32 or tlse.dtype != torch.float32 or lse.shape != q.shape[:3] \
             or tlse.shape != q.shape[:3]:
         raise ValueError("attn_fwd_jvp_out: lse/tlse must be fp32 [B,H,N]")
     s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
-    prob = _problem(q, scale, clean_tangent_zero)
+    prob = _problem(q, scale, clean_tangent_zero, token_major_out)
     st = _lib.lib().caj_attn_fwd_jvp(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
                                      ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)),
                                      ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(to.data_ptr()),
@@ -111,7 +118,7 @@ def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optiona
 
 
 def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
-                 clean_tangent_zero: bool = False):
+                 clean_tangent_zero: bool = False, token_major_out: bool = False):
     """Returns (o, to, lse, tlse). See the module docstring and attn_fwd_jvp_out.
 
     With CPU tensors the library's host-buffer entry point runs the call: it
@@ -120,12 +127,17 @@ def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
     in pinned host memory; pinned inputs copy fastest."""
     if q.is_cuda:
         ins = [q, k, v, tq, tk, tv]
-        o = torch.empty_like(q)
-        to = torch.empty_like(q)
+        B, H, N, D = q.shape
+        out_shape = (B, N, H, D) if token_major_out else (B, H, N, D)
+        o = torch.empty(out_shape, dtype=q.dtype, device=q.device)
+        to = torch.empty(out_shape, dtype=q.dtype, device=q.device)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
         tlse = torch.empty_like(lse)
-        attn_fwd_jvp_out(*ins, mask, o, to, lse, tlse, scale=scale, clean_tangent_zero=clean_tangent_zero)
+        attn_fwd_jvp_out(*ins, mask, o, to, lse, tlse, scale=scale, clean_tangent_zero=clean_tangent_zero,
+                         token_major_out=token_major_out)
         return o, to, lse, tlse
+    if token_major_out:
+        raise ValueError("attn_fwd_jvp: host tensors take the head-major output layout only")
     ins = (q, k, v, tq, tk, tv)
     for t in ins:
         if t.is_cuda or not t.is_contiguous():
@@ -152,6 +164,42 @@ def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
     _lib.check(st, "caj_attn_fwd_jvp_host")
     stream.synchronize()
     return o, to, lse, tlse
+
+
+def out_proj_jvp(x, tx, w, bias=None, out=None):
+    """Output projection in primal-tangent form (see include/causaljvp.h):
+    y = x W^T + bias, ty = tx W^T.
+
+    x, tx: [..., K] bf16 CUDA tensors (e.g. the attention output [B, N, H, D]
+    from attn_fwd_jvp(..., token_major_out=True), K = H*D); w: [C, K] bf16;
+    bias: [C] bf16 or None. Returns (y, ty) of shape [..., C]."""
+    C, K = w.shape
+    # rows of K elements: [..., K] or, for the token-major attention output, [..., H, D]
+    if x.shape[-1] == K:
+        lead = tuple(x.shape[:-1])
+    elif x.dim() >= 2 and x.shape[-2] * x.shape[-1] == K:
+        lead = tuple(x.shape[:-2])
+    else:
+        raise ValueError("out_proj_jvp: x's rows must hold the weight's K elements")
+    if tx.shape != x.shape or (bias is not None and tuple(bias.shape) != (C,)):
+        raise ValueError("out_proj_jvp: shape mismatch")
+    for t in (x, tx, w) + ((bias,) if bias is not None else ()):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16):
+            raise ValueError("out_proj_jvp: tensors must be contiguous bf16 CUDA tensors")
+    M = x.numel() // K
+    if out is None:
+        out = (torch.empty((M, C), dtype=torch.bfloat16, device=x.device),
+               torch.empty((M, C), dtype=torch.bfloat16, device=x.device))
+    y, ty = out
+    shape = _lib.LinearShapeC(M, K, C)
+    s = torch.cuda.current_stream(x.device).cuda_stream
+    st = _lib.lib().caj_out_proj_jvp(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(tx.data_ptr()),
+                                     ctypes.c_void_p(w.data_ptr()),
+                                     ctypes.c_void_p(bias.data_ptr() if bias is not None else 0),
+                                     ctypes.byref(shape), ctypes.c_void_p(y.data_ptr()),
+                                     ctypes.c_void_p(ty.data_ptr()), ctypes.c_void_p(s))
+    _lib.check(st, "caj_out_proj_jvp")
+    return y.view(*lead, C), ty.view(*lead, C)
 
 
 def qk_norm_rope_jvp(xq, xk, xv, txq, txk, txv, gq, gk, rope_cos, rope_sin, H: int,

@@ -17,8 +17,12 @@ EXPORTED = [
     "caj_status_string", "caj_last_cuda_error", "caj_validate_mask", "caj_visible_pairs",
     "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
     "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
-    "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host",
+    "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host", "caj_out_proj_jvp",
 ]
+
+
+class LinearShapeC(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int32), ("C", ctypes.c_int32)]
 
 
 class MaskDescC(ctypes.Structure):
@@ -33,6 +37,7 @@ class ProblemC(ctypes.Structure):
 
 
 CAJ_FLAG_CLEAN_TANGENT_ZERO = 1
+CAJ_FLAG_TOKEN_MAJOR_OUT = 2
 
 
 class PrologueShapeC(ctypes.Structure):
@@ -96,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.caj_attn_fwd_jvp_host.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC)] + \
             [vp] * 5 + [ctypes.c_size_t, vp]
         L.caj_attn_fwd_jvp_host.restype = ctypes.c_int
+        L.caj_out_proj_jvp.argtypes = [vp] * 4 + [ctypes.POINTER(LinearShapeC), vp, vp, vp]
+        L.caj_out_proj_jvp.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

@@ -3,6 +3,7 @@
 // include/causaljvp.h for the contract of every entry point.
 #include "causaljvp.h"
 
+#include <cublasLt.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -122,6 +123,82 @@ uint64_t wait_timeout_ns() {
 
 namespace {
 
+// ------------------------------------------------ output projection (cuBLASLt)
+// y = x W^T (+ bias), ty = tx W^T: two plain bf16 GEMMs with fp32
+// accumulation, the bias fused as cuBLASLt's epilogue. Row-major y[M][C] is the
+// column-major C x M matrix W (C x K) times x^T (K x M): A = w stored K x C
+// (transposed), B = x stored K x M, D = y stored C x M. No workspace, so
+// nothing is allocated per call; the handle is created once per process.
+caj_status lt_fail(cublasStatus_t s) {
+  std::snprintf(g_cuda_msg, sizeof g_cuda_msg, "cublasLt status %d", int(s));
+  return CAJ_ERR_CUDA;
+}
+
+cublasStatus_t lt_handle(cublasLtHandle_t *h) {
+  static std::mutex mu;
+  static cublasLtHandle_t handle = nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!handle) {
+    cublasStatus_t s = cublasLtCreate(&handle);
+    if (s != CUBLAS_STATUS_SUCCESS) return s;
+  }
+  *h = handle;
+  return CUBLAS_STATUS_SUCCESS;
+}
+
+cublasStatus_t lt_gemm(cublasLtHandle_t lt, const void *a_w, const void *b_x, void *d_y,
+                       const void *bias, int64_t M, int64_t K, int64_t C, cudaStream_t s) {
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  cublasStatus_t r = cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F);
+  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
+  if (r == CUBLAS_STATUS_SUCCESS)
+    r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta));
+  if (r == CUBLAS_STATUS_SUCCESS)
+    r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb));
+  if (r == CUBLAS_STATUS_SUCCESS && bias) {
+    const cublasLtEpilogue_t ep = CUBLASLT_EPILOGUE_BIAS;
+    const cudaDataType_t bt = CUDA_R_16BF;
+    r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_EPILOGUE, &ep, sizeof(ep));
+    if (r == CUBLAS_STATUS_SUCCESS)
+      r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_BIAS_POINTER, &bias, sizeof(bias));
+    if (r == CUBLAS_STATUS_SUCCESS)
+      r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_BIAS_DATA_TYPE, &bt, sizeof(bt));
+  }
+  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, K, C, K);
+  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, K, M, K);
+  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatrixLayoutCreate(&ld, CUDA_R_16BF, C, M, C);
+  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatmulPreferenceCreate(&pref);
+  const size_t no_workspace = 0;
+  if (r == CUBLAS_STATUS_SUCCESS)
+    r = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &no_workspace,
+                                             sizeof(no_workspace));
+  cublasLtMatmulHeuristicResult_t heur{};
+  int found = 0;
+  if (r == CUBLAS_STATUS_SUCCESS)
+    r = cublasLtMatmulAlgoGetHeuristic(lt, op, la, lb, ld, ld, pref, 1, &heur, &found);
+  if (r == CUBLAS_STATUS_SUCCESS && found == 0) r = CUBLAS_STATUS_NOT_SUPPORTED;
+  const float one = 1.f, zero = 0.f;
+  if (r == CUBLAS_STATUS_SUCCESS)
+    r = cublasLtMatmul(lt, op, &one, a_w, la, b_x, lb, &zero, d_y, ld, d_y, ld, &heur.algo, nullptr, 0, s);
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (ld) cublasLtMatrixLayoutDestroy(ld);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return r;
+}
+
+caj_status out_proj_gemms(const void *x, const void *tx, const void *w, const void *bias, int64_t M,
+                          int64_t K, int64_t C, void *y, void *ty, cudaStream_t s) {
+  cublasLtHandle_t lt = nullptr;
+  cublasStatus_t r = lt_handle(&lt);
+  if (r == CUBLAS_STATUS_SUCCESS) r = lt_gemm(lt, w, x, y, bias, M, K, C, s);        // primal
+  if (r == CUBLAS_STATUS_SUCCESS) r = lt_gemm(lt, w, tx, ty, nullptr, M, K, C, s);   // tangent
+  return r == CUBLAS_STATUS_SUCCESS ? CAJ_OK : lt_fail(r);
+}
+
 // Shape, dtype, flag and mask checks shared by the device and host forms of
 // the forward.
 caj_status validate_fwd(const caj_problem *prob, const caj_mask_desc *mask, caj::MaskGeom *g) {
@@ -130,7 +207,8 @@ caj_status validate_fwd(const caj_problem *prob, const caj_mask_desc *mask, caj:
   if (!geom_from_desc(mask, g) || g->N != prob->N) return CAJ_ERR_INVALID_ARG;
   if (prob->dtype != CAJ_DTYPE_F32 && prob->dtype != CAJ_DTYPE_BF16) return CAJ_ERR_INVALID_ARG;
   if (!(prob->scale >= 0.f) || std::isinf(prob->scale)) return CAJ_ERR_INVALID_ARG;
-  if (prob->flags & ~int32_t(CAJ_FLAG_CLEAN_TANGENT_ZERO)) return CAJ_ERR_INVALID_ARG;
+  if (prob->flags & ~int32_t(CAJ_FLAG_CLEAN_TANGENT_ZERO | CAJ_FLAG_TOKEN_MAJOR_OUT))
+    return CAJ_ERR_INVALID_ARG;
   if ((prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) && !mask->tf_layout) return CAJ_ERR_INVALID_ARG;
   if (prob->D != 64 && prob->D != 128) return CAJ_ERR_UNSUPPORTED;
   const int64_t BH = int64_t(prob->B) * prob->H;
@@ -297,6 +375,7 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
     p.geom = g;
     p.BH = int32_t(BH);
     p.scale = scale;
+    p.out_heads = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? prob->H : 0;
     cudaError_t e = caj::launch_fwd_jvp_simt_f32(p, prob->D, s);
     return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
   }
@@ -326,6 +405,7 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   p.timeout_ns = wait_timeout_ns();
   p.fault_mode = g_fault_mode.load();
   p.tile_kind = caj::kTilesAll;
+  p.out_heads = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? prob->H : 0;
   // Launch order: query tiles by decreasing number of key tiles (ties: later first).
   std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
   for (int32_t t = 0; t < n_qtiles; ++t) {
@@ -381,6 +461,8 @@ caj_status caj_attn_fwd_jvp_host(const void *q, const void *k, const void *v, co
   caj::MaskGeom g;
   caj_status st = validate_fwd(prob, mask, &g);
   if (st != CAJ_OK) return st;
+  // head chunks are copied as contiguous blocks: head-major outputs only
+  if (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) return CAJ_ERR_INVALID_ARG;
   HostWorkspace w;
   if (!host_workspace(prob, &w) || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       workspace_bytes < w.total)
@@ -444,6 +526,20 @@ caj_status caj_attn_fwd_jvp_host(const void *q, const void *k, const void *v, co
   if (kst != CAJ_OK) return kst;
   if (!good) return cuda_fail(e);
   return je == cudaSuccess ? CAJ_OK : cuda_fail(je);
+}
+
+caj_status caj_out_proj_jvp(const void *x, const void *tx, const void *w, const void *bias,
+                            const caj_linear_shape *shape, void *y, void *ty, void *stream) {
+  if (!shape || shape->M <= 0 || shape->K <= 0 || shape->C <= 0) return CAJ_ERR_INVALID_ARG;
+  if (shape->K % 8 || shape->C % 8) return CAJ_ERR_UNSUPPORTED;  // 16-byte rows
+  const void *ptrs[5] = {x, tx, w, y, ty};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
+  if (bias && !aligned16(bias)) return CAJ_ERR_INVALID_ARG;
+  caj_status st = check_device();
+  if (st != CAJ_OK) return st;
+  return out_proj_gemms(x, tx, w, bias, shape->M, shape->K, shape->C, y, ty,
+                        static_cast<cudaStream_t>(stream));
 }
 
 caj_status caj_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv, const void *txq,

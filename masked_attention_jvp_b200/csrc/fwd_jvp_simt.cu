@@ -113,8 +113,8 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_jvp_simt_f32_kernel(const Sim
 
   const float inv_l = 1.f / l_run;
   const float mu = r_run * inv_l;
-  float *O = static_cast<float *>(p.o) + head + size_t(qi) * D;
-  float *TO = static_cast<float *>(p.to) + head + size_t(qi) * D;
+  float *O = static_cast<float *>(p.o) + out_row(bh, qi, N, p.out_heads, D);
+  float *TO = static_cast<float *>(p.to) + out_row(bh, qi, N, p.out_heads, D);
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
     const float ov = oacc[e] * inv_l;

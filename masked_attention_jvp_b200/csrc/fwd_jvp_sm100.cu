@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv_l = 1.f / l_tot;
         const float mu = r_tot * inv_l;
         const bool store = q < p.geom.N;
-        const size_t rowoff = (size_t(bh) * p.geom.N + (store ? q : 0)) * D;
+        const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
         uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
         uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
 #pragma unroll 1
@@ -944,7 +944,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float w0 = f0 / l_tot, w1 = f1 / l_tot;
         const bool store = q < p.geom.N;
-        const size_t rowoff = (size_t(bh) * p.geom.N + (store ? q : 0)) * D;
+        const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
         uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
         uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
         // warpgroup g writes output columns [g D/2, (g+1) D/2)

@@ -46,6 +46,7 @@ struct Sm100Params {
   uint64_t timeout_ns;   // bounded-wait limit
   int32_t fault_mode;    // test hook: 1 = skip the query-tile copies
   int32_t tile_kind;     // TileKind: the query tiles this launch covers
+  int32_t out_heads;     // H when O, tO are token-major [B, N, H, D]; 0: [B, H, N, D]
   uint16_t qtile_order[kMaxQTiles];  // heaviest query tiles first
 };
 
@@ -56,7 +57,17 @@ struct SimtParams {
   MaskGeom geom;
   int32_t BH;
   float scale;
+  int32_t out_heads;  // H when O, tO are token-major [B, N, H, D]; 0: [B, H, N, D]
 };
+
+// Element offset of output row q of head bh (= b H + h): [B, H, N, D] when
+// out_heads == 0, else token-major [B, N, H, D] with H = out_heads (the input
+// layout of the output projection).
+__host__ __device__ inline size_t out_row(int32_t bh, int32_t q, int32_t N, int32_t out_heads, int D) {
+  if (out_heads == 0) return (size_t(bh) * N + q) * D;
+  const int32_t b = bh / out_heads, h = bh % out_heads;
+  return ((size_t(b) * N + q) * out_heads + h) * D;
+}
 
 struct PrologueParams {
   const void *xq, *xk, *xv, *txq, *txk, *txv;  // [B, N, H*D] bf16

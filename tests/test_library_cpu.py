@@ -255,3 +255,33 @@ def test_key_tile_schedule_matches_brute_force(mask, bk, bq):
         assert n == len(tiles)
         want = sorted({i // bq for j in range(k0, k1) for i in range(N) if oracle.visible(mask, i, j)})
         assert tiles == want, (mask, k0, k1, bk, bq)
+
+
+def test_out_proj_validation_launches_nothing():
+    vp = ctypes.c_void_p
+    L = _lib.lib()
+    INV, UNS = _lib.CAJ_ERR_INVALID_ARG, _lib.CAJ_ERR_UNSUPPORTED
+
+    def call(M=64, K=128, C=256, x=0x1000, bias=0, y=0x2000):
+        shape = _lib.LinearShapeC(M, K, C)
+        return L.caj_out_proj_jvp(vp(x), vp(x), vp(x), vp(bias), ctypes.byref(shape), vp(y), vp(y), vp(0))
+
+    assert call(M=0) == INV                  # no rows
+    assert call(K=0) == INV
+    assert call(K=100) == UNS                # rows not whole 16-byte units
+    assert call(C=36) == UNS
+    assert call(x=0) == INV                  # null input
+    assert call(x=0x1008) == INV             # misaligned input
+    assert call(bias=0x3004) == INV          # misaligned bias
+    assert L.caj_out_proj_jvp(vp(1), vp(1), vp(1), vp(0), None, vp(1), vp(1), vp(0)) == INV
+
+
+def test_token_major_flag_validation():
+    P, M = _lib.ProblemC, _lib.MaskDescC
+    bf, tm, ctz = _lib.CAJ_DTYPE_BF16, _lib.CAJ_FLAG_TOKEN_MAJOR_OUT, _lib.CAJ_FLAG_CLEAN_TANGENT_ZERO
+    assert _call(prob=P(1, 2, 64, 64, bf, 0.0, tm)) != _lib.CAJ_ERR_INVALID_ARG      # accepted
+    assert _call(prob=P(1, 2, 128, 64, bf, 0.0, tm | ctz), mask=M(16, 1, 4, 1)) != _lib.CAJ_ERR_INVALID_ARG
+    assert _call(prob=P(1, 2, 64, 64, bf, 0.0, 8)) == _lib.CAJ_ERR_INVALID_ARG       # unknown bit
+    # the host-buffer form copies head-major chunks only
+    _, need = _ws_bytes(P(1, 2, 64, 64, bf, 0.0))
+    assert _host_call(0x100000, need, prob=P(1, 2, 64, 64, bf, 0.0, tm)) == _lib.CAJ_ERR_INVALID_ARG
