@@ -42,7 +42,7 @@ KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struc
 PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
 BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
 # {(workload, sources_sha256): dram bytes read + written per launch}
-MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "fa7da86b1ef90280"): 1428828928 + 390922752}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "333eb4c43a802a97"): 1427503872 + 390638592}
 PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241276160 + 1150380544}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
 BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "97e98721674f6154"):
