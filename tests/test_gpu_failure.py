@@ -44,3 +44,33 @@ def test_fault_hook_rejects_unknown_modes():
     L = _lib.lib()
     assert L.caj_debug_set_fault(7) == _lib.CAJ_ERR_INVALID_ARG
     assert L.caj_debug_set_fault(0) == _lib.CAJ_OK
+
+
+def test_clean_tangent_zero_kernels_time_out_too():
+    """Both kernels of the clean-tangent-zero path (the JVP kernel on the noisy
+    query tile, the primal-only kernel on the clean one) bound their waits the
+    same way."""
+    L = _lib.lib()
+    from masked_attention_jvp_b200.workloads import zero_clean_tangents
+    w = Workload("fault_ctz", 1, 1, 128, MaskDesc(64, 1, 2, 1), torch.bfloat16, seed=6)  # L = 128
+    ins = make_inputs(w, "cuda")
+    zero_clean_tangents(w, *ins[3:])
+    caj.device_status()
+    assert L.caj_set_wait_timeout_ms(100.0) == _lib.CAJ_OK
+    assert L.caj_debug_set_fault(1) == _lib.CAJ_OK
+    try:
+        caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=True)
+        with pytest.raises(caj.CajError) as err:
+            caj.device_status()
+        assert err.value.status == _lib.CAJ_ERR_DEVICE_TIMEOUT
+        assert L.caj_last_device_error_code() & 0xFF00 == 0x100
+    finally:
+        L.caj_debug_set_fault(0)
+        L.caj_set_wait_timeout_ms(0.0)
+    caj.device_status()
+    o, to, lse, tlse = caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=True)
+    caj.device_status()
+    ro, rto, rlse, rtlse = oracle.attn_fwd_jvp(*[t.cpu() for t in ins], w.mask)
+    rel = lambda a, b: float(np.linalg.norm(a - b) / np.linalg.norm(b))
+    assert rel(o.float().cpu().numpy(), ro) <= 1e-2
+    assert rel(to.float().cpu().numpy(), rto) <= 1e-2
