@@ -79,10 +79,12 @@ typedef struct {
  * guarantees that tq, tk and tv are exactly zero on the clean half (token
  * rows < L). In TF-sCM the clean context has zero tangent and only the noisy
  * branch follows the teacher velocity (Causal-rCM section 3.1.2, the paragraph
- * after eq. 17). The kernel then skips every product that vanishes: query tiles
+ * after eq. 17). The call then skips every product that vanishes: query tiles
  * of clean rows compute only the primal (tO = 0, tLSE = 0), and key tiles of
- * clean tokens skip Q tK^T and P tV. With the guarantee the results equal the
- * dense definition; without it they do not.
+ * clean tokens skip Q tK^T and P tV. It runs as two kernel launches on
+ * `stream`, one per kind of query tile (tiles with a noisy row, then tiles of
+ * clean rows). With the guarantee the results equal the dense definition;
+ * without it they do not.
  */
 /*
  * CAJ_FLAG_TOKEN_MAJOR_OUT: o and to are written token-major, [B, N, H, D]
@@ -101,9 +103,10 @@ typedef enum { CAJ_FLAG_CLEAN_TANGENT_ZERO = 1, CAJ_FLAG_TOKEN_MAJOR_OUT = 2 } c
  * Supported: D in {64, 128}; dtype BF16 (tensor-core path, fp32 accumulation)
  * or F32 (CUDA-core fp32 path); N == n_frames*tokens_per_frame*(tf_layout?2:1);
  * B*H <= 65535; N <= 1048576.
- * Returns CAJ_OK once the kernel is enqueued, CAJ_ERR_INVALID_ARG /
- * CAJ_ERR_UNSUPPORTED without launching, or CAJ_ERR_CUDA if the launch failed.
- * Device-side bounded-wait failures are reported by caj_last_device_status.
+ * Returns CAJ_OK once the kernel(s) are enqueued on `stream` (asynchronous),
+ * CAJ_ERR_INVALID_ARG / CAJ_ERR_UNSUPPORTED without launching, or
+ * CAJ_ERR_CUDA if a launch failed. Device-side bounded-wait failures are
+ * reported by caj_last_device_status.
  */
 caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v,
                             const void *tq, const void *tk, const void *tv,
