@@ -279,3 +279,19 @@ def test_clean_tangent_zero_needs_teacher_forcing_layout():
     ins = make_inputs(w, "cuda")
     with pytest.raises(caj.CajError):
         caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=True)
+
+
+def test_clean_tangent_zero_repeated_calls_are_bitwise_identical():
+    """Both clean-tangent-zero kernels are deterministic (in the primal kernel
+    the two softmax warpgroups finish different tiles; their epilogues must
+    still see every value product)."""
+    from masked_attention_jvp_b200.workloads import zero_clean_tangents
+    w = Workload("ctzdet", 1, 4, 128, MaskDesc(200, 2, 6, 1), torch.bfloat16, seed=21)
+    ins = make_inputs(w, "cuda")
+    zero_clean_tangents(w, *ins[3:])
+    first = caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=True)
+    for _ in range(3):
+        again = caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=True)
+        for x, y in zip(first, again):
+            assert torch.equal(x, y)
+    caj.device_status()
