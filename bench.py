@@ -348,6 +348,42 @@ def bench_backward(w, ins, o, lse, steps, peaks):
             "executed_products_tflop": round(14 * w.D * pairs / 1e12, 3)}
 
 
+# ------------------------------------------------- clean-tangent-zero forward
+def bench_ctz(w, ins, steps, fl):
+    """The same workload as TF-sCM feeds it: the clean half's tangents are zero
+    and the call skips the products that vanish (two launches per call). The
+    value is dense-equivalent (12 D flops per visible pair) and, separately,
+    per needed product."""
+    import masked_attention_jvp_b200 as caj
+    from masked_attention_jvp_b200.workloads import zero_clean_tangents
+    tq, tk, tv = (t.clone() for t in ins[3:])
+    zero_clean_tangents(w, tq, tk, tv)
+    args = ins[:3] + [tq, tk, tv]
+    o, to = torch.empty_like(ins[0]), torch.empty_like(ins[0])
+    lse = torch.empty(ins[0].shape[:3], dtype=torch.float32, device=ins[0].device)
+    tlse = torch.empty_like(lse)
+
+    def call():
+        caj.attn_fwd_jvp_out(*args, w.mask, o, to, lse, tlse, scale=w.scale, clean_tangent_zero=True)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    caj.device_status()
+    ms = e0.elapsed_time(e1) / steps
+    L = w.mask.n_frames * w.mask.tokens_per_frame
+    return {"ms": round(ms, 4), "dense_equivalent_tflops": round(fl / (ms / 1e3) / 1e12, 2),
+            "needed_products_tflop": round(ctz_product_flops(w) / 1e12, 3),
+            "needed_products_tflops": round(ctz_product_flops(w) / (ms / 1e3) / 1e12, 2),
+            "kernels": ["fwd_jvp_sm100_kernel<128, kTilesNoisyCTZ>", "fwd_primal_sm100_kernel<128>"],
+            "gpu_launches": steps * (2 if L >= 128 else 1)}
+
+
 # ------------------------------------------------------------ output projection
 def bench_out_proj(w, dev, steps, peaks):
     """Output projection in primal-tangent form on the workload's tokens:
@@ -491,6 +527,8 @@ def bench_gpu(args, rank, world, local_rank):
         line["gpu_launches_prologue"] = args.steps
     if not args.no_out_proj and not args.clean_tangent_zero:
         line["out_proj"] = bench_out_proj(w, dev, args.steps, peaks)
+    if w.mask.tf_layout and not args.clean_tangent_zero and not args.no_ctz:
+        line["clean_tangent_zero"] = bench_ctz(w, ins, args.steps, fl)
     if args.clean_tangent_zero:
         # one launch for the query tiles with a noisy row, one for the clean ones
         L = w.mask.n_frames * w.mask.tokens_per_frame
@@ -566,6 +604,8 @@ def main():
     ap.add_argument("--no-prologue", action="store_true", help="skip the prologue kernel's measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward kernels' measurement")
     ap.add_argument("--no-out-proj", action="store_true", help="skip the output projection's measurement")
+    ap.add_argument("--no-ctz", action="store_true",
+                    help="skip the clean-tangent-zero sub-measurement (teacher-forcing workloads)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (small cases for ncu section captures)")
     ap.add_argument("--clean-tangent-zero", action="store_true",
