@@ -42,7 +42,7 @@ KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struc
 PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
 BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
 # {(workload, sources_sha256): dram bytes read + written per launch}
-MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "333eb4c43a802a97"): 1427503872 + 390638592}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "1879393c29d6e8ff"): 1426112768 + 390586368}
 PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241276160 + 1150380544}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
 BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "97e98721674f6154"):
@@ -415,6 +415,56 @@ def bench_out_proj(w, dev, steps, peaks):
             "frac": round(tf / peak, 4)}
 
 
+def bench_cp_scatter(w, ins, steps, fl):
+    """One rank's attention under P-way Ulysses context parallelism, emulated on
+    this GPU: the rank's H/P heads over the whole sequence, written once to a
+    plain [B, H/P, N, D] output and once scattered to the P sequence slices
+    [B, H, N/P, D] (the epilogue doing the output all-to-all; the slices are
+    local here, peer memory on a multi-GPU run). The two timings show what the
+    scattered store costs in the kernel. No NVLink traffic is measured."""
+    import masked_attention_jvp_b200 as caj
+    P = next((p for p in (4, 2) if w.H % p == 0 and w.N % p == 0), None)
+    if P is None:
+        return None
+    Hp, Ls = w.H // P, w.N // P
+    mine = [x[:, :Hp].contiguous() for x in ins]
+    dev = mine[0].device
+    o = torch.empty(w.B, Hp, w.N, w.D, dtype=w.dtype, device=dev)
+    to = torch.empty_like(o)
+    lse = torch.empty(w.B, Hp, w.N, dtype=torch.float32, device=dev)
+    tlse = torch.empty_like(lse)
+    so = [torch.empty(w.B, w.H, Ls, w.D, dtype=w.dtype, device=dev) for _ in range(P)]
+    sto = [torch.empty_like(t) for t in so]
+    sl = [torch.empty(w.B, w.H, Ls, dtype=torch.float32, device=dev) for _ in range(P)]
+    stl = [torch.empty_like(t) for t in sl]
+    plain = lambda: caj.attn_fwd_jvp_out(*mine, w.mask, o, to, lse, tlse, scale=w.scale)
+    scatter = lambda: caj.attn_fwd_jvp_scatter(*mine, w.mask, so, sto, sl, stl, head_base=0, scale=w.scale)
+    res = {"ranks": P, "heads_per_rank": Hp, "slice_rows": Ls}
+    # interleaved rounds, so that clock drift under the power cap hits both alike
+    fns = {"plain": plain, "scatter": scatter}
+    per_round = max(2, steps // 4)
+    times = {k: [] for k in fns}
+    for fn in fns.values():
+        for _ in range(3):
+            fn()
+    torch.cuda.synchronize()
+    for _ in range(4):
+        for name, fn in fns.items():
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(per_round):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            times[name].append(e0.elapsed_time(e1) / per_round)
+    for name, t in times.items():
+        ms = statistics.median(t)
+        res[f"ms_{name}"] = round(ms, 4)
+        res[f"tflops_{name}"] = round(fl / P / (ms / 1e3) / 1e12, 2)
+    res["scatter_over_plain"] = round(res["ms_scatter"] / res["ms_plain"], 4)
+    return res
+
+
 # ------------------------------------------------------------------ GPU arm
 def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
     """Same metric through the public API from pinned host buffers: every step
@@ -527,6 +577,11 @@ def bench_gpu(args, rank, world, local_rank):
         line["gpu_launches_prologue"] = args.steps
     if not args.no_out_proj and not args.clean_tangent_zero:
         line["out_proj"] = bench_out_proj(w, dev, args.steps, peaks)
+    if not args.no_cp_scatter and not args.clean_tangent_zero:
+        cp = bench_cp_scatter(w, ins, args.steps, fl)
+        if cp is not None:
+            line["cp_scatter"] = cp
+            line["gpu_launches_cp_scatter"] = 2 * 4 * max(2, args.steps // 4)
     if w.mask.tf_layout and not args.clean_tangent_zero and not args.no_ctz:
         line["clean_tangent_zero"] = bench_ctz(w, ins, args.steps, fl)
     if args.clean_tangent_zero:
@@ -604,6 +659,8 @@ def main():
     ap.add_argument("--no-prologue", action="store_true", help="skip the prologue kernel's measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward kernels' measurement")
     ap.add_argument("--no-out-proj", action="store_true", help="skip the output projection's measurement")
+    ap.add_argument("--no-cp-scatter", action="store_true",
+                    help="skip the context-parallel output-scatter measurement")
     ap.add_argument("--no-ctz", action="store_true",
                     help="skip the clean-tangent-zero sub-measurement (teacher-forcing workloads)")
     ap.add_argument("--heads", type=int, default=None,

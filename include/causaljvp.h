@@ -115,6 +115,56 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v,
                             void *stream);
 
 /*
+ * Context-parallel form of caj_attn_fwd_jvp, with the output all-to-all done by
+ * the kernel's epilogue. Causal-rCM trains with flattened Ulysses context
+ * parallelism (section 3.2.1, "Parallelism"; section 3.2.2, "JVP Ulysses CP").
+ * Each of P ranks holds N/P tokens of every head. An all-to-all gives each rank
+ * H/P heads over the whole sequence. Local attention runs, and the outputs and
+ * their tangents return through a second all-to-all. The tangents follow the
+ * same route as their primals.
+ * Here the second all-to-all is not a separate collective: each output row is
+ * written directly into the buffers of the rank that owns its sequence slice.
+ *   in : q, k, v, tq, tk, tv   this rank's heads over the whole sequence,
+ *                              [B,H,N,D] of prob->dtype (H = heads of this rank)
+ *   dst->shards                P, 1..CAJ_MAX_SHARDS; N must be a multiple of P
+ *   dst->head_base             global index of this call's head 0
+ *   dst->heads_total           heads of each slice buffer, at least
+ *                              head_base + H
+ *   dst->o[r], dst->to[r]      slice r (token rows [r N/P, (r+1) N/P)):
+ *                              [B, heads_total, N/P, D] of prob->dtype, or
+ *                              [B, N/P, heads_total, D] with
+ *                              CAJ_FLAG_TOKEN_MAJOR_OUT; 16-byte aligned
+ *   dst->lse[r], dst->tlse[r]  slice r: [B, heads_total, N/P] fp32
+ * Only the rows of this call's heads are written. The other heads' rows in
+ * the slice buffers are left as they are. Values and rounding equal those of
+ * caj_attn_fwd_jvp on the same inputs.
+ * On a multi-GPU run the slice buffers of the other ranks are their device
+ * memory mapped into this process: CUDA IPC or symmetric memory, with peer
+ * access enabled. The kernel writes them with plain stores over NVLink.
+ * The library does not synchronise with the peers. Before the call the caller
+ * makes sure that no rank still reads the slice buffers. After it, the caller
+ * orders every rank's reads after all P calls, e.g. with a barrier on the
+ * stream. The buffers are owned by the caller.
+ * Returns as caj_attn_fwd_jvp. CAJ_ERR_INVALID_ARG is also returned for a null
+ * dst, a shard count or head range out of bounds, or a null or misaligned
+ * slice pointer.
+ */
+#define CAJ_MAX_SHARDS 8
+typedef struct {
+  int32_t shards;
+  int32_t head_base;
+  int32_t heads_total;
+  void *o[CAJ_MAX_SHARDS];
+  void *to[CAJ_MAX_SHARDS];
+  float *lse[CAJ_MAX_SHARDS];
+  float *tlse[CAJ_MAX_SHARDS];
+} caj_seq_scatter;
+caj_status caj_attn_fwd_jvp_scatter(const void *q, const void *k, const void *v,
+                                    const void *tq, const void *tk, const void *tv,
+                                    const caj_problem *prob, const caj_mask_desc *mask,
+                                    const caj_seq_scatter *dst, void *stream);
+
+/*
  * Host-buffer form of caj_attn_fwd_jvp: the same operation, with the inputs
  * and outputs in host memory. The heads are split into at most 16 chunks.
  * Three things run at once on three streams: the copy of chunk c's six inputs

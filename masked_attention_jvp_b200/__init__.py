@@ -28,7 +28,7 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -164,6 +164,56 @@ def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
     _lib.check(st, "caj_attn_fwd_jvp_host")
     stream.synchronize()
     return o, to, lse, tlse
+
+
+def attn_fwd_jvp_scatter(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, head_base: int = 0,
+                         scale: Optional[float] = None, stream: Optional[torch.cuda.Stream] = None,
+                         clean_tangent_zero: bool = False, token_major_out: bool = False) -> None:
+    """Forward + JVP whose output rows go straight to their sequence slice.
+
+    q..tv: [B, H, N, D] CUDA tensors, this call's H heads over the whole packed
+    sequence. o, to, lse, tlse: lists of P tensors, entry r the buffers of
+    sequence slice r (token rows [r N/P, (r+1) N/P)): o[r], to[r] are
+    [B, Ht, N/P, D] ([B, N/P, Ht, D] with token_major_out), lse[r], tlse[r]
+    fp32 [B, Ht, N/P], where Ht >= head_base + H is the heads of a slice. Head h
+    of the call fills head head_base + h of every slice; other heads are left
+    as they are. In Ulysses context parallelism entry r is rank r's memory
+    mapped into this process, and the call is the attention plus the output
+    all-to-all (include/causaljvp.h, caj_attn_fwd_jvp_scatter: the caller
+    orders the ranks around it)."""
+    ins = (q, k, v, tq, tk, tv)
+    P = len(o)
+    if not 1 <= P <= _lib.MAX_SHARDS or not (len(to) == len(lse) == len(tlse) == P):
+        raise ValueError(f"attn_fwd_jvp_scatter: o, to, lse, tlse need one entry per slice (1..{_lib.MAX_SHARDS})")
+    for t in ins:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("attn_fwd_jvp_scatter: q..tv must be contiguous CUDA tensors")
+    if q.dtype not in _DTYPES or any(t.dtype != q.dtype or t.shape != q.shape for t in ins):
+        raise ValueError("attn_fwd_jvp_scatter: q..tv must share one shape and dtype (bf16 or fp32)")
+    B, H, N, D = q.shape
+    if N % P:
+        raise ValueError(f"attn_fwd_jvp_scatter: sequence length {N} is not a multiple of {P} slices")
+    Ht = (o[0].shape[2] if token_major_out else o[0].shape[1]) if o[0].dim() == 4 else -1
+    Ls = N // P
+    out_shape = (B, Ls, Ht, D) if token_major_out else (B, Ht, Ls, D)
+    for r in range(P):
+        for t in (o[r], to[r]):
+            if t.dtype != q.dtype or tuple(t.shape) != out_shape or not t.is_contiguous():
+                raise ValueError(f"attn_fwd_jvp_scatter: slice {r} output must be contiguous {out_shape}")
+        for t in (lse[r], tlse[r]):
+            if t.dtype != torch.float32 or tuple(t.shape) != (B, Ht, Ls) or not t.is_contiguous():
+                raise ValueError(f"attn_fwd_jvp_scatter: slice {r} lse/tlse must be contiguous fp32 {(B, Ht, Ls)}")
+    dst = _lib.SeqScatterC()
+    dst.shards, dst.head_base, dst.heads_total = P, int(head_base), Ht
+    for r in range(P):
+        dst.o[r], dst.to[r] = o[r].data_ptr(), to[r].data_ptr()
+        dst.lse[r], dst.tlse[r] = lse[r].data_ptr(), tlse[r].data_ptr()
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    prob = _problem(q, scale, clean_tangent_zero, token_major_out)
+    st = _lib.lib().caj_attn_fwd_jvp_scatter(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
+                                             ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)),
+                                             ctypes.byref(dst), ctypes.c_void_p(s))
+    _lib.check(st, "caj_attn_fwd_jvp_scatter")
 
 
 def out_proj_jvp(x, tx, w, bias=None, out=None):

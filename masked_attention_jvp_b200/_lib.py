@@ -18,7 +18,17 @@ EXPORTED = [
     "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
     "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
     "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host", "caj_out_proj_jvp",
+    "caj_attn_fwd_jvp_scatter",
 ]
+
+
+MAX_SHARDS = 8  # CAJ_MAX_SHARDS
+
+
+class SeqScatterC(ctypes.Structure):
+    _fields_ = [("shards", ctypes.c_int32), ("head_base", ctypes.c_int32), ("heads_total", ctypes.c_int32),
+                ("o", ctypes.c_void_p * MAX_SHARDS), ("to", ctypes.c_void_p * MAX_SHARDS),
+                ("lse", ctypes.c_void_p * MAX_SHARDS), ("tlse", ctypes.c_void_p * MAX_SHARDS)]
 
 
 class LinearShapeC(ctypes.Structure):
@@ -103,6 +113,9 @@ def lib() -> ctypes.CDLL:
         L.caj_attn_fwd_jvp_host.restype = ctypes.c_int
         L.caj_out_proj_jvp.argtypes = [vp] * 4 + [ctypes.POINTER(LinearShapeC), vp, vp, vp]
         L.caj_out_proj_jvp.restype = ctypes.c_int
+        L.caj_attn_fwd_jvp_scatter.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC),
+                                                ctypes.POINTER(SeqScatterC), vp]
+        L.caj_attn_fwd_jvp_scatter.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

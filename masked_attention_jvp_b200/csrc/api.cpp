@@ -348,38 +348,26 @@ int32_t caj_ktile_query_tiles(const caj_mask_desc *mask, int32_t k0, int32_t k1,
   return n;
 }
 
-caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const void *tq,
-                            const void *tk, const void *tv, const caj_problem *prob,
-                            const caj_mask_desc *mask, void *o, void *to, float *lse, float *tlse,
-                            void *stream) {
-  const void *ins[6] = {q, k, v, tq, tk, tv};
-  for (const void *p : ins)
-    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
-  if (!o || !to || !aligned16(o) || !aligned16(to)) return CAJ_ERR_INVALID_ARG;
-  if (!lse || !tlse || !aligned4(lse) || !aligned4(tlse)) return CAJ_ERR_INVALID_ARG;
-  caj::MaskGeom g;
-  caj_status st = validate_fwd(prob, mask, &g);
-  if (st != CAJ_OK) return st;
+namespace {
+
+// Launches the forward + JVP of a validated problem on `s`, the output rows
+// placed by `out`.
+caj_status fwd_launch(const void *const in[6], const caj_problem *prob, const caj::MaskGeom &g,
+                      const caj::OutMap &out, cudaStream_t s) {
+  const void *q = in[0], *k = in[1], *v = in[2], *tq = in[3], *tk = in[4], *tv = in[5];
   const int64_t BH = int64_t(prob->B) * prob->H;
-
-  st = check_device();
-  if (st != CAJ_OK) return st;
-
   const float scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt(float(prob->D));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   if (prob->dtype == CAJ_DTYPE_F32) {
     caj::SimtParams p{};
     p.q = q; p.k = k; p.v = v; p.tq = tq; p.tk = tk; p.tv = tv;
-    p.o = o; p.to = to; p.lse = lse; p.tlse = tlse;
+    p.out = out;
     p.geom = g;
     p.BH = int32_t(BH);
     p.scale = scale;
-    p.out_heads = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? prob->H : 0;
     cudaError_t e = caj::launch_fwd_jvp_simt_f32(p, prob->D, s);
     return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
   }
-
   const int32_t n_qtiles = (prob->N + caj::kBlockM - 1) / caj::kBlockM;
   if (n_qtiles > caj::kMaxQTiles) return CAJ_ERR_UNSUPPORTED;
   EncodeTiledFn enc = get_encode_tiled();
@@ -396,7 +384,7 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
              encode_map(enc, &p.tm_v, v, int(BH), N, D, caj::kBlockN) &&
              encode_map(enc, &p.tm_tv, tv, int(BH), N, D, caj::kBlockN);
   if (!okm) return cuda_fail(cudaErrorInvalidValue);
-  p.o = o; p.to = to; p.lse = lse; p.tlse = tlse;
+  p.out = out;
   p.geom = g;
   p.BH = int32_t(BH);
   p.n_qtiles = n_qtiles;
@@ -405,7 +393,6 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   p.timeout_ns = wait_timeout_ns();
   p.fault_mode = g_fault_mode.load();
   p.tile_kind = caj::kTilesAll;
-  p.out_heads = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? prob->H : 0;
   // Launch order: query tiles by decreasing number of key tiles (ties: later first).
   std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
   for (int32_t t = 0; t < n_qtiles; ++t) {
@@ -440,6 +427,72 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
 
   cudaError_t e = caj::launch_fwd_jvp_sm100(p, D, s);
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const void *tq,
+                            const void *tk, const void *tv, const caj_problem *prob,
+                            const caj_mask_desc *mask, void *o, void *to, float *lse, float *tlse,
+                            void *stream) {
+  const void *ins[6] = {q, k, v, tq, tk, tv};
+  for (const void *p : ins)
+    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
+  if (!o || !to || !aligned16(o) || !aligned16(to)) return CAJ_ERR_INVALID_ARG;
+  if (!lse || !tlse || !aligned4(lse) || !aligned4(tlse)) return CAJ_ERR_INVALID_ARG;
+  caj::MaskGeom g;
+  caj_status st = validate_fwd(prob, mask, &g);
+  if (st != CAJ_OK) return st;
+  st = check_device();
+  if (st != CAJ_OK) return st;
+
+  caj::OutMap out{};
+  out.o[0] = o; out.to[0] = to; out.lse[0] = lse; out.tlse[0] = tlse;
+  out.shards = 1;
+  out.shard_len = prob->N;
+  out.heads = out.heads_total = prob->H;
+  out.head_base = 0;
+  out.token_major = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? 1 : 0;
+  return fwd_launch(ins, prob, g, out, static_cast<cudaStream_t>(stream));
+}
+
+static_assert(CAJ_MAX_SHARDS == caj::kMaxShards, "slice count of the public and kernel output maps");
+
+caj_status caj_attn_fwd_jvp_scatter(const void *q, const void *k, const void *v, const void *tq,
+                                    const void *tk, const void *tv, const caj_problem *prob,
+                                    const caj_mask_desc *mask, const caj_seq_scatter *dst,
+                                    void *stream) {
+  const void *ins[6] = {q, k, v, tq, tk, tv};
+  for (const void *p : ins)
+    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
+  caj::MaskGeom g;
+  caj_status st = validate_fwd(prob, mask, &g);
+  if (st != CAJ_OK) return st;
+  if (!dst || dst->shards < 1 || dst->shards > CAJ_MAX_SHARDS || prob->N % dst->shards)
+    return CAJ_ERR_INVALID_ARG;
+  if (dst->head_base < 0 || dst->heads_total < prob->H || dst->head_base > dst->heads_total - prob->H)
+    return CAJ_ERR_INVALID_ARG;
+  for (int32_t r = 0; r < dst->shards; ++r) {
+    if (!dst->o[r] || !dst->to[r] || !aligned16(dst->o[r]) || !aligned16(dst->to[r]))
+      return CAJ_ERR_INVALID_ARG;
+    if (!dst->lse[r] || !dst->tlse[r] || !aligned4(dst->lse[r]) || !aligned4(dst->tlse[r]))
+      return CAJ_ERR_INVALID_ARG;
+  }
+  st = check_device();
+  if (st != CAJ_OK) return st;
+
+  caj::OutMap out{};
+  for (int32_t r = 0; r < dst->shards; ++r) {
+    out.o[r] = dst->o[r]; out.to[r] = dst->to[r];
+    out.lse[r] = dst->lse[r]; out.tlse[r] = dst->tlse[r];
+  }
+  out.shards = dst->shards;
+  out.shard_len = prob->N / dst->shards;
+  out.heads = prob->H;
+  out.head_base = dst->head_base;
+  out.heads_total = dst->heads_total;
+  out.token_major = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? 1 : 0;
+  return fwd_launch(ins, prob, g, out, static_cast<cudaStream_t>(stream));
 }
 
 caj_status caj_attn_fwd_jvp_host_workspace(const caj_problem *prob, size_t *bytes) {

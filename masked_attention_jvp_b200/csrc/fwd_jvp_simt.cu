@@ -34,7 +34,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kWarps * 32) fwd_jvp_simt_f32_kernel(const SimtParams p) {
+__global__ void __launch_bounds__(kWarps * 32) fwd_jvp_simt_f32_kernel(const __grid_constant__ SimtParams p) {
   constexpr int PER = D / 32;  // elements of D owned by each lane
   __shared__ float4 sq[kWarps][D / 4], stq[kWarps][D / 4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -113,8 +113,9 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_jvp_simt_f32_kernel(const Sim
 
   const float inv_l = 1.f / l_run;
   const float mu = r_run * inv_l;
-  float *O = static_cast<float *>(p.o) + out_row(bh, qi, N, p.out_heads, D);
-  float *TO = static_cast<float *>(p.to) + out_row(bh, qi, N, p.out_heads, D);
+  const OutRow dst = out_row(p.out, bh, qi);
+  float *O = static_cast<float *>(p.out.o[dst.shard]) + dst.row * D;
+  float *TO = static_cast<float *>(p.out.to[dst.shard]) + dst.row * D;
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
     const float ov = oacc[e] * inv_l;
@@ -122,8 +123,8 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_jvp_simt_f32_kernel(const Sim
     TO[lane + 32 * e] = fmaf(tacc[e], inv_l, -mu * ov);
   }
   if (lane == 0) {
-    p.lse[gid] = m_run + logf(l_run);
-    p.tlse[gid] = mu;
+    p.out.lse[dst.shard][dst.stat] = m_run + logf(l_run);
+    p.out.tlse[dst.shard][dst.stat] = mu;
   }
 }
 

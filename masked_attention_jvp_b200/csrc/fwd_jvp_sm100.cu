@@ -564,9 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv_l = 1.f / l_tot;
         const float mu = r_tot * inv_l;
         const bool store = q < p.geom.N;
-        const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
-        uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
-        uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
+        const OutRow dst = out_row(p.out, bh, store ? q : 0);
+        uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.o[dst.shard]) + dst.row * D);
+        uint4 *torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.to[dst.shard]) + dst.row * D);
 #pragma unroll 1
         for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
           uint32_t ro[32], rt[32];
@@ -590,9 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (store && g == 0) {
-          const size_t ri = size_t(bh) * p.geom.N + q;
-          p.lse[ri] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
-          p.tlse[ri] = mu;
+          p.out.lse[dst.shard][dst.stat] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+          p.out.tlse[dst.shard][dst.stat] = mu;
         }
       }
     }
@@ -944,9 +943,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float w0 = f0 / l_tot, w1 = f1 / l_tot;
         const bool store = q < p.geom.N;
-        const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
-        uint4 *orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
-        uint4 *torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
+        const OutRow dst = out_row(p.out, bh, store ? q : 0);
+        uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.o[dst.shard]) + dst.row * D);
+        uint4 *torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.to[dst.shard]) + dst.row * D);
         // warpgroup g writes output columns [g D/2, (g+1) D/2)
 #pragma unroll 1
         for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
@@ -971,9 +970,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (store && g == 0) {
-          const size_t ri = size_t(bh) * p.geom.N + q;
-          p.lse[ri] = (m + __log2f(l_tot)) * 0.69314718055994530942f;
-          p.tlse[ri] = 0.f;
+          p.out.lse[dst.shard][dst.stat] = (m + __log2f(l_tot)) * 0.69314718055994530942f;
+          p.out.tlse[dst.shard][dst.stat] = 0.f;
         }
       }
     }

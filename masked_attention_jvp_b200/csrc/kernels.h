@@ -34,10 +34,48 @@ enum TileKind : int32_t {
   kTilesCleanCTZ = 2,  // clean-tangent-zero: tiles of clean rows only (primal only)
 };
 
+// Largest number of sequence slices one output map scatters to: the GPUs of
+// one NVSwitch domain.
+constexpr int kMaxShards = 8;
+
+// Where the output rows of a launch go. The packed sequence of N rows is cut
+// into `shards` equal slices of `shard_len` rows; slice r lives in buffers
+// o[r], to[r], lse[r], tlse[r]. In context-parallel (Ulysses) attention slice r
+// belongs to rank r and those buffers are its memory, reached over NVLink, so
+// the epilogue itself performs the output all-to-all. Head h of the launch
+// (bh = b * heads + h) is head head_base + h of the heads_total heads each slice
+// holds. O, tO: [B, heads_total, shard_len, D], or [B, shard_len, heads_total, D]
+// when token_major (the input layout of the output projection). LSE, tLSE:
+// [B, heads_total, shard_len]. One slice with head_base = 0 and
+// heads_total = heads is the plain [B, H, N, D] output.
+struct OutMap {
+  void *o[kMaxShards], *to[kMaxShards];
+  float *lse[kMaxShards], *tlse[kMaxShards];
+  int32_t shards, shard_len;
+  int32_t heads, head_base, heads_total;
+  int32_t token_major;
+};
+
+// Output row q of head bh: its slice, its O/tO row (in units of D elements)
+// and its LSE/tLSE element.
+struct OutRow {
+  int32_t shard;
+  size_t row, stat;
+};
+
+__host__ __device__ inline OutRow out_row(const OutMap &m, int32_t bh, int32_t q) {
+  const int32_t b = bh / m.heads, h = m.head_base + bh % m.heads;
+  const int32_t r = q / m.shard_len, ql = q - r * m.shard_len;
+  OutRow o;
+  o.shard = r;
+  o.stat = (size_t(b) * m.heads_total + h) * m.shard_len + ql;
+  o.row = m.token_major ? (size_t(b) * m.shard_len + ql) * m.heads_total + h : o.stat;
+  return o;
+}
+
 struct Sm100Params {
   CUtensorMap tm_q, tm_tq, tm_k, tm_tk, tm_v, tm_tv;  // 3-D maps over [B*H, N, D]
-  void *o, *to;          // [B*H, N, D] bf16
-  float *lse, *tlse;     // [B*H, N]
+  OutMap out;            // where O, tO (bf16) and LSE, tLSE rows go
   MaskGeom geom;
   int32_t BH;
   int32_t n_qtiles;
@@ -46,28 +84,16 @@ struct Sm100Params {
   uint64_t timeout_ns;   // bounded-wait limit
   int32_t fault_mode;    // test hook: 1 = skip the query-tile copies
   int32_t tile_kind;     // TileKind: the query tiles this launch covers
-  int32_t out_heads;     // H when O, tO are token-major [B, N, H, D]; 0: [B, H, N, D]
   uint16_t qtile_order[kMaxQTiles];  // heaviest query tiles first
 };
 
 struct SimtParams {
   const void *q, *k, *v, *tq, *tk, *tv;
-  void *o, *to;
-  float *lse, *tlse;
+  OutMap out;  // where O, tO (fp32) and LSE, tLSE rows go
   MaskGeom geom;
   int32_t BH;
   float scale;
-  int32_t out_heads;  // H when O, tO are token-major [B, N, H, D]; 0: [B, H, N, D]
 };
-
-// Element offset of output row q of head bh (= b H + h): [B, H, N, D] when
-// out_heads == 0, else token-major [B, N, H, D] with H = out_heads (the input
-// layout of the output projection).
-__host__ __device__ inline size_t out_row(int32_t bh, int32_t q, int32_t N, int32_t out_heads, int D) {
-  if (out_heads == 0) return (size_t(bh) * N + q) * D;
-  const int32_t b = bh / out_heads, h = bh % out_heads;
-  return ((size_t(b) * N + q) * out_heads + h) * D;
-}
 
 struct PrologueParams {
   const void *xq, *xk, *xv, *txq, *txk, *txv;  // [B, N, H*D] bf16

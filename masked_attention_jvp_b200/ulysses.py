@@ -9,11 +9,16 @@ follow exactly the communication pattern of their primals, the local attention
 is the masked attention JVP kernel, and the output tangent returns through the
 same all-to-all as the output.
 
-Here the six inputs travel in one all-to-all and the four outputs in two (the
-bf16 pair O, tO and the fp32 pair LSE, tLSE). The mask needs no translation,
-because the local call sees the whole packed sequence. Collectives go through
-torch.distributed (NCCL over NVLink on GPUs). All arithmetic is in the local
-kernel.
+Here the six inputs travel in one all-to-all. The four outputs return one of
+two ways:
+  - two all-to-alls (the bf16 pair O, tO and the fp32 pair LSE, tLSE), or
+  - with fused_output=True, no collective at all: the kernel's epilogue writes
+    every output row into the symmetric-memory slice buffers of the rank that
+    owns its tokens (caj_attn_fwd_jvp_scatter), over NVLink, and two
+    stream-ordered barriers fence the writes.
+The mask needs no translation, because the local call sees the whole packed
+sequence. Collectives go through torch.distributed (NCCL over NVLink on GPUs).
+All arithmetic is in the local kernel.
 """
 from __future__ import annotations
 
@@ -60,9 +65,57 @@ def head_to_seq(y: torch.Tensor, group=None) -> torch.Tensor:
     return recv.permute(1, 2, 0, 3, 4, 5).reshape(S, B, P * Hp, Ls, E)
 
 
+class SliceBuffers:
+    """This rank's output slice in symmetric memory, mapped on every rank.
+
+    One allocation holds O, tO [B, H, Ls, D] and LSE, tLSE [B, H, Ls] fp32
+    (regions 256-byte aligned). o[r], to[r], lse[r], tlse[r] view rank r's copy:
+    rank r's device memory, reached over NVLink for r != this rank."""
+
+    def __init__(self, B: int, H: int, Ls: int, D: int, dtype: torch.dtype, device, group=None):
+        import torch.distributed._symmetric_memory as symm_mem
+
+        def up(x):
+            return (x + 255) // 256 * 256
+
+        es = torch.empty((), dtype=dtype).element_size()
+        n_out, n_st = B * H * Ls * D, B * H * Ls
+        offs = [0, up(n_out * es), 2 * up(n_out * es), 2 * up(n_out * es) + up(n_st * 4)]
+        total = offs[3] + up(n_st * 4)
+        self.key = (B, H, Ls, D, dtype, torch.device(device))
+        self.buf = symm_mem.empty(total, dtype=torch.uint8, device=device)
+        self.handle = symm_mem.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
+        self.rank, self.world = self.handle.rank, self.handle.world_size
+        hd = self.handle
+
+        def view(r, off, shape, dt):
+            return hd.get_buffer(r, shape, dt, off // torch.empty((), dtype=dt).element_size())
+
+        P = self.world
+        self.o = [view(r, offs[0], (B, H, Ls, D), dtype) for r in range(P)]
+        self.to = [view(r, offs[1], (B, H, Ls, D), dtype) for r in range(P)]
+        self.lse = [view(r, offs[2], (B, H, Ls), torch.float32) for r in range(P)]
+        self.tlse = [view(r, offs[3], (B, H, Ls), torch.float32) for r in range(P)]
+
+    def barrier(self, timeout_ms: int = 10000):
+        """Stream-ordered barrier over the group's ranks."""
+        self.handle.barrier(channel=0, timeout_ms=timeout_ms)
+
+
+_slice_buffers = {}
+
+
+def _get_slice_buffers(B, H, Ls, D, dtype, device, group) -> SliceBuffers:
+    key = (B, H, Ls, D, dtype, torch.device(device), id(group))
+    sb = _slice_buffers.get(key)
+    if sb is None:
+        sb = _slice_buffers[key] = SliceBuffers(B, H, Ls, D, dtype, device, group)
+    return sb
+
+
 def ulysses_attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None, group=None,
                          clean_tangent_zero: bool = False,
-                         local_fn: Optional[Callable] = None):
+                         local_fn: Optional[Callable] = None, fused_output: bool = False):
     """Context-parallel forward + JVP.
 
     q..tv: this rank's sequence shard, [B, H, N/P, D], where shard r holds
@@ -71,13 +124,45 @@ def ulysses_attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = Non
     [B, H, N/P]. local_fn(q, k, v, tq, tk, tv, mask, scale=..., clean_tangent_zero=...)
     computes attention on the head-sharded full sequence. It defaults to the
     fused kernel (masked_attention_jvp_b200.attn_fwd_jvp).
+
+    fused_output=True (CUDA tensors, the fused kernel): the output all-to-all
+    is done by the kernel's epilogue, which stores each row into the
+    symmetric-memory slice buffer of its owner (see SliceBuffers). The
+    returned tensors are copies, so the slice buffers are free for the next
+    call once every rank has passed its first barrier.
     """
+    ins = torch.stack([q, k, v, tq, tk, tv])
+    if fused_output:
+        if local_fn is not None:
+            raise ValueError("fused_output runs the fused kernel; local_fn does not apply")
+        return _ulysses_fused_output(ins, mask, scale, group, clean_tangent_zero)
     if local_fn is None:
         from . import attn_fwd_jvp as local_fn
-    ins = torch.stack([q, k, v, tq, tk, tv])
     full = seq_to_head(ins, group)
     o, to, lse, tlse = local_fn(*full.unbind(0), mask, scale=scale,
                                 clean_tangent_zero=clean_tangent_zero)
     out = head_to_seq(torch.stack([o, to]), group)
     stats = head_to_seq(torch.stack([lse, tlse]).unsqueeze(-1), group).squeeze(-1)
     return out[0], out[1], stats[0], stats[1]
+
+
+def _ulysses_fused_output(ins, mask, scale, group, clean_tangent_zero):
+    from . import attn_fwd_jvp_scatter
+    P = _world(group)
+    _, B, H, Ls, D = ins.shape
+    full = seq_to_head(ins, group)
+    Hp = H // P
+    sb = _get_slice_buffers(B, H, Ls, D, ins.dtype, ins.device, group)
+    # every rank has copied its previous results out of its slice buffer
+    sb.barrier()
+    attn_fwd_jvp_scatter(*full.unbind(0), mask, sb.o, sb.to, sb.lse, sb.tlse, head_base=sb.rank * Hp,
+                         scale=scale, clean_tangent_zero=clean_tangent_zero)
+    # every rank's rows have landed in this rank's slice buffer
+    sb.barrier()
+    me = sb.rank
+    return sb.o[me].clone(), sb.to[me].clone(), sb.lse[me].clone(), sb.tlse[me].clone()
+
+
+def release_slice_buffers() -> None:
+    """Drops the cached slice buffers (before the process group goes away)."""
+    _slice_buffers.clear()

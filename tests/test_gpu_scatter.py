@@ -1,0 +1,91 @@
+"""The forward + JVP with its output all-to-all in the epilogue
+(caj_attn_fwd_jvp_scatter), on one GPU: P ranks of Ulysses context parallelism
+(Causal-rCM section 3.2.1 "Parallelism", section 3.2.2 "JVP Ulysses CP") are
+emulated as P launches, launch r computing heads [r H/P, (r+1) H/P) over the
+whole sequence and storing every row into the slice buffer of the token's
+owner. The P slice buffers are local here; on a multi-GPU run they are the
+ranks' memory and the same stores cross NVLink. The launches only store, they
+never wait on one another. After all P launches slice r must equal rows
+[r N/P, (r+1) N/P) of the direct call, bit for bit, for every head."""
+import pytest
+import torch
+
+import masked_attention_jvp_b200 as caj
+from masked_attention_jvp_b200.workloads import MaskDesc, make_inputs, small, zero_clean_tangents
+
+pytestmark = pytest.mark.gpu
+
+bf, f32 = torch.bfloat16, torch.float32
+
+# name, B, H, D, mask, dtype, P, clean_tangent_zero, token_major
+CASES = [
+    ("tf_p2", 1, 4, 128, MaskDesc(100, 1, 4, 1), bf, 2, False, False),          # N 800, slices of 400
+    ("infer_d64_p4_ragged", 2, 4, 64, MaskDesc(75, 1, 8, 0), bf, 4, False, False),  # slices of 150: tiles straddle
+    ("tf_ctz_p4", 1, 8, 128, MaskDesc(100, 1, 4, 1), bf, 4, True, False),       # both CTZ launches scatter
+    ("tf_chunk_tokmajor_p2", 1, 4, 128, MaskDesc(60, 3, 6, 1), bf, 2, False, True),
+    ("tf_ctz_tokmajor_p8", 1, 8, 64, MaskDesc(40, 1, 8, 1), bf, 8, True, True),  # 8 slices of 80 rows
+    ("fp32_p2", 1, 2, 64, MaskDesc(16, 1, 4, 0), f32, 2, False, False),          # CUDA-core path
+    ("tf_p1", 1, 2, 128, MaskDesc(50, 1, 3, 1), bf, 1, False, False),            # one slice: plain output
+]
+
+
+def _slices(B, H, Ls, D, dtype, P, token_major):
+    shp = (B, Ls, H, D) if token_major else (B, H, Ls, D)
+    full = lambda s, dt: [torch.full(s, float("nan"), dtype=dt, device="cuda") for _ in range(P)]
+    return full(shp, dtype), full(shp, dtype), full((B, H, Ls), f32), full((B, H, Ls), f32)
+
+
+def _rows(t, rows, token_major):
+    return t[:, rows] if token_major else t[:, :, rows]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_scatter_equals_direct_call(case):
+    name, B, H, D, mask, dtype, P, ctz, tm = case
+    w = small(name, B, H, D, mask, dtype, seed=31)
+    ins = make_inputs(w, "cuda")
+    if ctz:
+        zero_clean_tangents(w, *ins[3:])
+    direct = caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=ctz, token_major_out=tm)
+    N, Hp = w.N, H // P
+    Ls = N // P
+    o, to, lse, tlse = _slices(B, H, Ls, D, dtype, P, tm)
+    for r in range(P):  # emulated rank r: its heads, every slice
+        mine = [x[:, r * Hp:(r + 1) * Hp].contiguous() for x in ins]
+        caj.attn_fwd_jvp_scatter(*mine, w.mask, o, to, lse, tlse, head_base=r * Hp,
+                                 clean_tangent_zero=ctz, token_major_out=tm)
+    torch.cuda.synchronize()
+    for r in range(P):
+        rows = slice(r * Ls, (r + 1) * Ls)
+        assert torch.equal(o[r], _rows(direct[0], rows, tm)), (name, r, "o")
+        assert torch.equal(to[r], _rows(direct[1], rows, tm)), (name, r, "to")
+        assert torch.equal(lse[r], direct[2][:, :, rows]), (name, r, "lse")
+        assert torch.equal(tlse[r], direct[3][:, :, rows]), (name, r, "tlse")
+
+
+def test_scatter_writes_only_its_own_heads():
+    B, H, D, P = 1, 4, 128, 2
+    w = small("own_heads", B, H, D, MaskDesc(100, 1, 4, 1), bf, seed=32)
+    ins = make_inputs(w, "cuda")
+    direct = caj.attn_fwd_jvp(*ins, w.mask)
+    Ls, Hp = w.N // P, H // P
+    o, to, lse, tlse = _slices(B, H, Ls, D, bf, P, False)
+    mine = [x[:, Hp:].contiguous() for x in ins]  # rank 1 alone
+    caj.attn_fwd_jvp_scatter(*mine, w.mask, o, to, lse, tlse, head_base=Hp)
+    torch.cuda.synchronize()
+    for r in range(P):
+        rows = slice(r * Ls, (r + 1) * Ls)
+        for got, want in ((o[r], direct[0]), (to[r], direct[1]), (lse[r], direct[2]), (tlse[r], direct[3])):
+            assert torch.equal(got[:, Hp:], want[:, Hp:, rows])
+            assert torch.isnan(got[:, :Hp].float()).all()  # rank 0's heads untouched
+
+
+def test_scatter_rejects_bad_slices():
+    w = small("bad", 1, 2, 64, MaskDesc(16, 1, 4, 0), bf, seed=33)
+    ins = make_inputs(w, "cuda")
+    o, to, lse, tlse = _slices(1, 2, 21, 64, bf, 3, False)
+    with pytest.raises(ValueError):  # 64 rows do not split in 3
+        caj.attn_fwd_jvp_scatter(*ins, w.mask, o, to, lse, tlse)
+    o, to, lse, tlse = _slices(1, 2, 32, 64, bf, 2, False)
+    with pytest.raises(caj.CajError):  # heads 1, 2 of a 2-head slice
+        caj.attn_fwd_jvp_scatter(*ins, w.mask, o, to, lse, tlse, head_base=1)

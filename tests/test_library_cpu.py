@@ -285,3 +285,43 @@ def test_token_major_flag_validation():
     # the host-buffer form copies head-major chunks only
     _, need = _ws_bytes(P(1, 2, 64, 64, bf, 0.0))
     assert _host_call(0x100000, need, prob=P(1, 2, 64, 64, bf, 0.0, tm)) == _lib.CAJ_ERR_INVALID_ARG
+
+
+def _scatter_call(shards=2, head_base=0, heads_total=4, prob=None, mask=None, o=0x20000, lse=0x30000,
+                  null_slice=None):
+    prob = prob or _lib.ProblemC(1, 2, 64, 64, _lib.CAJ_DTYPE_BF16, 0.0, 0)
+    mask = mask or _lib.MaskDescC(16, 1, 4, 0)
+    d = _lib.SeqScatterC()
+    d.shards, d.head_base, d.heads_total = shards, head_base, heads_total
+    for r in range(_lib.MAX_SHARDS):
+        step = 0 if r == null_slice else 1
+        d.o[r], d.to[r] = step * (o + 0x1000 * r), step * (o + 0x1000 * r + 0x800)
+        d.lse[r], d.tlse[r] = step * (lse + 0x1000 * r), step * (lse + 0x1000 * r + 0x800)
+    vp = ctypes.c_void_p
+    return _lib.lib().caj_attn_fwd_jvp_scatter(*[vp(0x10000)] * 6, ctypes.byref(prob), ctypes.byref(mask),
+                                               ctypes.byref(d), vp(0))
+
+
+def test_scatter_validation_launches_nothing():
+    P = _lib.ProblemC
+    bf, INV = _lib.CAJ_DTYPE_BF16, _lib.CAJ_ERR_INVALID_ARG
+    vp = ctypes.c_void_p
+    L = _lib.lib()
+    prob, mask = P(1, 2, 64, 64, bf, 0.0, 0), _lib.MaskDescC(16, 1, 4, 0)
+    assert L.caj_attn_fwd_jvp_scatter(*[vp(0x10000)] * 6, ctypes.byref(prob), ctypes.byref(mask),
+                                      None, vp(0)) == INV                    # no descriptor
+    assert _scatter_call(shards=0) == INV                                    # no slice
+    assert _scatter_call(shards=_lib.MAX_SHARDS + 1) == INV                  # more slices than the map holds
+    assert _scatter_call(shards=3) == INV                                    # 64 rows do not split in 3
+    assert _scatter_call(head_base=-1) == INV                                # head range below 0
+    assert _scatter_call(head_base=3, heads_total=4) == INV                  # heads 3, 4 of 4
+    assert _scatter_call(heads_total=1) == INV                               # fewer heads than the call
+    assert _scatter_call(o=0x20008) == INV                                   # misaligned O slice
+    assert _scatter_call(lse=0x30002) == INV                                 # misaligned LSE slice
+    assert _scatter_call(null_slice=1) == INV                                # a used slice is null
+    assert _scatter_call(shards=1, null_slice=1) != INV                      # an unused one may be
+    assert _scatter_call(prob=P(1, 2, 64, 64, bf, 0.0, 1)) == INV            # clean-tangent needs TF
+    assert _scatter_call(prob=P(1, 2, 64, 96, bf, 0.0)) == _lib.CAJ_ERR_UNSUPPORTED
+    for ok in (dict(shards=8, head_base=2), dict(shards=4, heads_total=2),
+               dict(prob=P(1, 2, 64, 64, bf, 0.0, _lib.CAJ_FLAG_TOKEN_MAJOR_OUT))):
+        assert _scatter_call(**ok) != INV, ok
