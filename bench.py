@@ -42,7 +42,7 @@ KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struc
 PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
 BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
 # {(workload, sources_sha256): dram bytes read + written per launch}
-MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "1879393c29d6e8ff"): 1426112768 + 390586368}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "3faf74fd960242a1"): 1429135872 + 390781696}
 PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241276160 + 1150380544}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
 BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "97e98721674f6154"):
@@ -577,13 +577,14 @@ def bench_gpu(args, rank, world, local_rank):
         line["gpu_launches_prologue"] = args.steps
     if not args.no_out_proj and not args.clean_tangent_zero:
         line["out_proj"] = bench_out_proj(w, dev, args.steps, peaks)
+    if w.mask.tf_layout and not args.clean_tangent_zero and not args.no_ctz:
+        line["clean_tangent_zero"] = bench_ctz(w, ins, args.steps, fl)
+    # last: it heats the GPU, and the legs above keep their earlier conditions
     if not args.no_cp_scatter and not args.clean_tangent_zero:
         cp = bench_cp_scatter(w, ins, args.steps, fl)
         if cp is not None:
             line["cp_scatter"] = cp
             line["gpu_launches_cp_scatter"] = 2 * 4 * max(2, args.steps // 4)
-    if w.mask.tf_layout and not args.clean_tangent_zero and not args.no_ctz:
-        line["clean_tangent_zero"] = bench_ctz(w, ins, args.steps, fl)
     if args.clean_tangent_zero:
         # one launch for the query tiles with a noisy row, one for the clean ones
         L = w.mask.n_frames * w.mask.tokens_per_frame

@@ -351,9 +351,10 @@ int32_t caj_ktile_query_tiles(const caj_mask_desc *mask, int32_t k0, int32_t k1,
 namespace {
 
 // Launches the forward + JVP of a validated problem on `s`, the output rows
-// placed by `out`.
+// placed by `out`: a one-slice output, or (scatter) the slices of a
+// context-parallel output.
 caj_status fwd_launch(const void *const in[6], const caj_problem *prob, const caj::MaskGeom &g,
-                      const caj::OutMap &out, cudaStream_t s) {
+                      const caj::OutMap &out, bool scatter, cudaStream_t s) {
   const void *q = in[0], *k = in[1], *v = in[2], *tq = in[3], *tk = in[4], *tv = in[5];
   const int64_t BH = int64_t(prob->B) * prob->H;
   const float scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt(float(prob->D));
@@ -384,7 +385,12 @@ caj_status fwd_launch(const void *const in[6], const caj_problem *prob, const ca
              encode_map(enc, &p.tm_v, v, int(BH), N, D, caj::kBlockN) &&
              encode_map(enc, &p.tm_tv, tv, int(BH), N, D, caj::kBlockN);
   if (!okm) return cuda_fail(cudaErrorInvalidValue);
-  p.out = out;
+  if (scatter) {
+    p.scatter = out;
+  } else {
+    p.o = out.o[0]; p.to = out.to[0]; p.lse = out.lse[0]; p.tlse = out.tlse[0];
+    p.out_heads = out.token_major ? prob->H : 0;
+  }
   p.geom = g;
   p.BH = int32_t(BH);
   p.n_qtiles = n_qtiles;
@@ -453,7 +459,7 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   out.heads = out.heads_total = prob->H;
   out.head_base = 0;
   out.token_major = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? 1 : 0;
-  return fwd_launch(ins, prob, g, out, static_cast<cudaStream_t>(stream));
+  return fwd_launch(ins, prob, g, out, false, static_cast<cudaStream_t>(stream));
 }
 
 static_assert(CAJ_MAX_SHARDS == caj::kMaxShards, "slice count of the public and kernel output maps");
@@ -492,7 +498,7 @@ caj_status caj_attn_fwd_jvp_scatter(const void *q, const void *k, const void *v,
   out.head_base = dst->head_base;
   out.heads_total = dst->heads_total;
   out.token_major = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? 1 : 0;
-  return fwd_launch(ins, prob, g, out, static_cast<cudaStream_t>(stream));
+  return fwd_launch(ins, prob, g, out, true, static_cast<cudaStream_t>(stream));
 }
 
 caj_status caj_attn_fwd_jvp_host_workspace(const caj_problem *prob, size_t *bytes) {

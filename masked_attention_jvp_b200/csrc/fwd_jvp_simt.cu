@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_jvp_simt_f32_kernel(const __g
 
   const float inv_l = 1.f / l_run;
   const float mu = r_run * inv_l;
-  const OutRow dst = out_row(p.out, bh, qi);
+  const OutRow dst = slice_row(p.out, bh, qi);
   float *O = static_cast<float *>(p.out.o[dst.shard]) + dst.row * D;
   float *TO = static_cast<float *>(p.out.to[dst.shard]) + dst.row * D;
 #pragma unroll

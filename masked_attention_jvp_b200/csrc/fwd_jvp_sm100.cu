@@ -201,7 +201,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // tiles have a kernel of their own (fwd_primal_sm100_kernel). Measured on the
 // TF frame-wise workload: one kernel branching on the kind of each tile took
 // 16.0 ms, the two specialised launches 12.0 ms.
-template <int D, int KIND>
+template <int D, int KIND, bool SCATTER>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {
   using C = Cfg<D>;
@@ -564,9 +564,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv_l = 1.f / l_tot;
         const float mu = r_tot * inv_l;
         const bool store = q < p.geom.N;
-        const OutRow dst = out_row(p.out, bh, store ? q : 0);
-        uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.o[dst.shard]) + dst.row * D);
-        uint4 *torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.to[dst.shard]) + dst.row * D);
+        uint4 *orow, *torow;
+        if constexpr (SCATTER) {
+          const OutRow dst = slice_row(p.scatter, bh, store ? q : 0);
+          orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.o[dst.shard]) + dst.row * D);
+          torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.to[dst.shard]) + dst.row * D);
+        } else {
+          const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
+          orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
+          torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
+        }
 #pragma unroll 1
         for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
           uint32_t ro[32], rt[32];
@@ -590,8 +597,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (store && g == 0) {
-          p.out.lse[dst.shard][dst.stat] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
-          p.out.tlse[dst.shard][dst.stat] = mu;
+          const float lse = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+          if constexpr (SCATTER) {
+            const OutRow dst = slice_row(p.scatter, bh, q);
+            p.scatter.lse[dst.shard][dst.stat] = lse;
+            p.scatter.tlse[dst.shard][dst.stat] = mu;
+          } else {
+            const size_t ri = size_t(bh) * p.geom.N + q;
+            p.lse[ri] = lse;
+            p.tlse[ri] = mu;
+          }
         }
       }
     }
@@ -673,7 +688,7 @@ __device__ __forceinline__ PBarriers make_pbarriers(uint32_t base) {
   return b;
 }
 
-template <int D>
+template <int D, bool SCATTER>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_primal_sm100_kernel(const __grid_constant__ Sm100Params p) {
   using C = PCfg<D>;
@@ -943,9 +958,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float w0 = f0 / l_tot, w1 = f1 / l_tot;
         const bool store = q < p.geom.N;
-        const OutRow dst = out_row(p.out, bh, store ? q : 0);
-        uint4 *orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.o[dst.shard]) + dst.row * D);
-        uint4 *torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out.to[dst.shard]) + dst.row * D);
+        uint4 *orow, *torow;
+        if constexpr (SCATTER) {
+          const OutRow dst = slice_row(p.scatter, bh, store ? q : 0);
+          orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.o[dst.shard]) + dst.row * D);
+          torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.to[dst.shard]) + dst.row * D);
+        } else {
+          const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
+          orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
+          torow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.to) + rowoff);
+        }
         // warpgroup g writes output columns [g D/2, (g+1) D/2)
 #pragma unroll 1
         for (int c = g * (D / 2); c < (g + 1) * (D / 2); c += 32) {
@@ -970,8 +992,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (store && g == 0) {
-          p.out.lse[dst.shard][dst.stat] = (m + __log2f(l_tot)) * 0.69314718055994530942f;
-          p.out.tlse[dst.shard][dst.stat] = 0.f;
+          const float lse = (m + __log2f(l_tot)) * 0.69314718055994530942f;
+          if constexpr (SCATTER) {
+            const OutRow dst = slice_row(p.scatter, bh, q);
+            p.scatter.lse[dst.shard][dst.stat] = lse;
+            p.scatter.tlse[dst.shard][dst.stat] = 0.f;
+          } else {
+            const size_t ri = size_t(bh) * p.geom.N + q;
+            p.lse[ri] = lse;
+            p.tlse[ri] = 0.f;
+          }
         }
       }
     }
@@ -985,48 +1015,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool SCATTER>
 cudaError_t launch_primal_impl(const Sm100Params &p, cudaStream_t stream) {
   using C = PCfg<D>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_primal_sm100_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(fwd_primal_sm100_kernel<D, SCATTER>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
-  fwd_primal_sm100_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  fwd_primal_sm100_kernel<D, SCATTER><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <int D, int KIND>
+template <int D, int KIND, bool SCATTER>
 cudaError_t launch_impl(const Sm100Params &p, cudaStream_t stream) {
   using C = Cfg<D>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D, KIND>,
+    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D, KIND, SCATTER>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
-  fwd_jvp_sm100_kernel<D, KIND><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
+  fwd_jvp_sm100_kernel<D, KIND, SCATTER><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError();
+}
+
+// The scattering epilogue is an instantiation of its own: the one-slice
+// kernels keep their plain addressing. (One kernel for both, through the
+// slice map, measured 3-5% slower on the dense path under the power cap.)
+template <bool SCATTER>
+cudaError_t dispatch(const Sm100Params &p, int D, cudaStream_t stream) {
+  switch (p.tile_kind * 256 + D) {
+    case kTilesAll * 256 + 128: return launch_impl<128, kTilesAll, SCATTER>(p, stream);
+    case kTilesNoisyCTZ * 256 + 128: return launch_impl<128, kTilesNoisyCTZ, SCATTER>(p, stream);
+    case kTilesCleanCTZ * 256 + 128: return launch_primal_impl<128, SCATTER>(p, stream);
+    case kTilesAll * 256 + 64: return launch_impl<64, kTilesAll, SCATTER>(p, stream);
+    case kTilesNoisyCTZ * 256 + 64: return launch_impl<64, kTilesNoisyCTZ, SCATTER>(p, stream);
+    case kTilesCleanCTZ * 256 + 64: return launch_primal_impl<64, SCATTER>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream) {
-  switch (p.tile_kind * 256 + D) {
-    case kTilesAll * 256 + 128: return launch_impl<128, kTilesAll>(p, stream);
-    case kTilesNoisyCTZ * 256 + 128: return launch_impl<128, kTilesNoisyCTZ>(p, stream);
-    case kTilesCleanCTZ * 256 + 128: return launch_primal_impl<128>(p, stream);
-    case kTilesAll * 256 + 64: return launch_impl<64, kTilesAll>(p, stream);
-    case kTilesNoisyCTZ * 256 + 64: return launch_impl<64, kTilesNoisyCTZ>(p, stream);
-    case kTilesCleanCTZ * 256 + 64: return launch_primal_impl<64>(p, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  return p.scatter.shards > 0 ? dispatch<true>(p, D, stream) : dispatch<false>(p, D, stream);
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, uint32_t *out) {

@@ -63,7 +63,7 @@ struct OutRow {
   size_t row, stat;
 };
 
-__host__ __device__ inline OutRow out_row(const OutMap &m, int32_t bh, int32_t q) {
+__host__ __device__ inline OutRow slice_row(const OutMap &m, int32_t bh, int32_t q) {
   const int32_t b = bh / m.heads, h = m.head_base + bh % m.heads;
   const int32_t r = q / m.shard_len, ql = q - r * m.shard_len;
   OutRow o;
@@ -73,9 +73,19 @@ __host__ __device__ inline OutRow out_row(const OutMap &m, int32_t bh, int32_t q
   return o;
 }
 
+// Element offset of output row q of head bh (= b H + h) in a one-slice output:
+// [B, H, N, D] when out_heads == 0, else token-major [B, N, H, D] with
+// H = out_heads. Equal to slice_row of the one-slice map, times D.
+__host__ __device__ inline size_t out_row(int32_t bh, int32_t q, int32_t N, int32_t out_heads, int D) {
+  if (out_heads == 0) return (size_t(bh) * N + q) * D;
+  const int32_t b = bh / out_heads, h = bh % out_heads;
+  return ((size_t(b) * N + q) * out_heads + h) * D;
+}
+
 struct Sm100Params {
   CUtensorMap tm_q, tm_tq, tm_k, tm_tk, tm_v, tm_tv;  // 3-D maps over [B*H, N, D]
-  OutMap out;            // where O, tO (bf16) and LSE, tLSE rows go
+  void *o, *to;          // one-slice output: [B*H, N, D] bf16
+  float *lse, *tlse;     // [B*H, N]
   MaskGeom geom;
   int32_t BH;
   int32_t n_qtiles;
@@ -84,7 +94,12 @@ struct Sm100Params {
   uint64_t timeout_ns;   // bounded-wait limit
   int32_t fault_mode;    // test hook: 1 = skip the query-tile copies
   int32_t tile_kind;     // TileKind: the query tiles this launch covers
+  int32_t out_heads;     // H when O, tO are token-major [B, N, H, D]; 0: [B, H, N, D]
   uint16_t qtile_order[kMaxQTiles];  // heaviest query tiles first
+  // Sequence slices of a context-parallel output. shards == 0: the launch
+  // writes the one-slice output above; otherwise the scattering
+  // instantiations write through this map and o, to, lse, tlse are unused.
+  OutMap scatter;
 };
 
 struct SimtParams {

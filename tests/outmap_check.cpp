@@ -1,11 +1,12 @@
-// Host check of the attention kernels' output map (caj::out_row in
+// Host check of the attention kernels' output map (caj::slice_row in
 // csrc/kernels.h), built and run by test_outmap_cpu.py. For every shape it
 // emulates the P launches of P-way Ulysses context parallelism (launch r holds
 // heads [r H/P, (r+1) H/P) over the whole sequence) and checks that each
 // (head, row) lands in slice q / (N/P) at the expected row of that slice's
 // [B, H, N/P, D] (or [B, N/P, H, D]) buffer and [B, H, N/P] statistics, in bounds,
-// with every row of every slice written exactly once. The plain one-slice map
-// must give the [B, H, N, D] addressing of a single call.
+// with every row of every slice written exactly once. The one-slice map must
+// give the addressing of a single call (caj::out_row, head-major and
+// token-major).
 #include <cstdio>
 #include <vector>
 
@@ -28,7 +29,7 @@ int main() {
               m.head_base = r0 * Hp; m.heads_total = H; m.token_major = tm;
               for (int bh = 0; bh < B * Hp; ++bh)
                 for (int q = 0; q < N; ++q) {
-                  const caj::OutRow d = caj::out_row(m, bh, q);
+                  const caj::OutRow d = caj::slice_row(m, bh, q);
                   if (d.shard < 0 || d.shard >= P || d.row >= lim || d.stat >= lim) { ++bad; continue; }
                   const int b = bh / Hp, h = r0 * Hp + bh % Hp, ql = q % Ls;
                   const size_t st = (size_t(b) * H + h) * Ls + ql;
@@ -47,12 +48,15 @@ int main() {
         m.shards = 1; m.shard_len = N; m.heads = H; m.heads_total = H;
         for (int bh = 0; bh < B * H; ++bh)
           for (int q = 0; q < N; ++q) {
-            caj::OutRow d = caj::out_row(m, bh, q);
+            const int D = 64;
+            caj::OutRow d = caj::slice_row(m, bh, q);
             bad += d.shard != 0 || d.stat != size_t(bh) * N + q || d.row != d.stat;
+            bad += d.row * D != caj::out_row(bh, q, N, 0, D);
             m.token_major = 1;
-            d = caj::out_row(m, bh, q);
+            d = caj::slice_row(m, bh, q);
             m.token_major = 0;
             bad += d.row != (size_t(bh / H) * N + q) * H + bh % H;
+            bad += d.row * D != caj::out_row(bh, q, N, H, D);
           }
       }
   std::printf("mismatches %ld\n", bad);
