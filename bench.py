@@ -42,7 +42,7 @@ KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struc
 PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
 BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
 # {(workload, sources_sha256): dram bytes read + written per launch}
-MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "3faf74fd960242a1"): 1429135872 + 390781696}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "89634e6b4f35b9e7"): 1431131648 + 390999296}
 PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241276160 + 1150380544}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
 BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "97e98721674f6154"):

@@ -201,6 +201,23 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // tiles have a kernel of their own (fwd_primal_sm100_kernel). Measured on the
 // TF frame-wise workload: one kernel branching on the kind of each tile took
 // 16.0 ms, the two specialised launches 12.0 ms.
+// The slice-map arithmetic of the scattering epilogues, kept out of line.
+// Inlined, it changed the register allocation of the kernels' main loop:
+// the scattering kernel then ran 4.7% slower than the plain one, against
+// 2.9% out of line (3 heads of the TF frame-wise workload, round-robin).
+__device__ __noinline__ void scatter_rows(const OutMap &m, int32_t bh, int32_t q, int D, uint4 **o,
+                                          uint4 **to) {
+  const OutRow dst = slice_row(m, bh, q);
+  *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(m.o[dst.shard]) + dst.row * D);
+  *to = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(m.to[dst.shard]) + dst.row * D);
+}
+
+__device__ __noinline__ void scatter_stats(const OutMap &m, int32_t bh, int32_t q, float lse, float tlse) {
+  const OutRow dst = slice_row(m, bh, q);
+  m.lse[dst.shard][dst.stat] = lse;
+  m.tlse[dst.shard][dst.stat] = tlse;
+}
+
 template <int D, int KIND, bool SCATTER>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {
@@ -566,9 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool store = q < p.geom.N;
         uint4 *orow, *torow;
         if constexpr (SCATTER) {
-          const OutRow dst = slice_row(p.scatter, bh, store ? q : 0);
-          orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.o[dst.shard]) + dst.row * D);
-          torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.to[dst.shard]) + dst.row * D);
+          scatter_rows(p.scatter, bh, store ? q : 0, D, &orow, &torow);
         } else {
           const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
           orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
@@ -599,9 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (store && g == 0) {
           const float lse = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
           if constexpr (SCATTER) {
-            const OutRow dst = slice_row(p.scatter, bh, q);
-            p.scatter.lse[dst.shard][dst.stat] = lse;
-            p.scatter.tlse[dst.shard][dst.stat] = mu;
+            scatter_stats(p.scatter, bh, q, lse, mu);
           } else {
             const size_t ri = size_t(bh) * p.geom.N + q;
             p.lse[ri] = lse;
@@ -960,9 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool store = q < p.geom.N;
         uint4 *orow, *torow;
         if constexpr (SCATTER) {
-          const OutRow dst = slice_row(p.scatter, bh, store ? q : 0);
-          orow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.o[dst.shard]) + dst.row * D);
-          torow = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.scatter.to[dst.shard]) + dst.row * D);
+          scatter_rows(p.scatter, bh, store ? q : 0, D, &orow, &torow);
         } else {
           const size_t rowoff = out_row(bh, store ? q : 0, p.geom.N, p.out_heads, D);
           orow = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + rowoff);
@@ -994,9 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (store && g == 0) {
           const float lse = (m + __log2f(l_tot)) * 0.69314718055994530942f;
           if constexpr (SCATTER) {
-            const OutRow dst = slice_row(p.scatter, bh, q);
-            p.scatter.lse[dst.shard][dst.stat] = lse;
-            p.scatter.tlse[dst.shard][dst.stat] = 0.f;
+            scatter_stats(p.scatter, bh, q, lse, 0.f);
           } else {
             const size_t ri = size_t(bh) * p.geom.N + q;
             p.lse[ri] = lse;
