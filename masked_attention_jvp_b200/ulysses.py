@@ -146,17 +146,25 @@ def ulysses_attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = Non
     return out[0], out[1], stats[0], stats[1]
 
 
-def _ulysses_fused_output(ins, mask, scale, group, clean_tangent_zero):
-    from . import attn_fwd_jvp_scatter
+def _ulysses_fused_output(ins, mask, scale, group, clean_tangent_zero, slices=None, scatter_fn=None):
+    """The fused-output path. `slices` (default: this group's SliceBuffers)
+    provides rank, o, to, lse, tlse and barrier(); `scatter_fn` (default: the
+    scattering kernel, attn_fwd_jvp_scatter) stores this rank's heads into
+    every slice. Both are replaceable so that the multi-rank control flow can
+    run on CPU ranks."""
     P = _world(group)
     _, B, H, Ls, D = ins.shape
+    if H % P:
+        raise ValueError(f"heads ({H}) must divide evenly over {P} ranks")
     full = seq_to_head(ins, group)
     Hp = H // P
-    sb = _get_slice_buffers(B, H, Ls, D, ins.dtype, ins.device, group)
+    sb = slices if slices is not None else _get_slice_buffers(B, H, Ls, D, ins.dtype, ins.device, group)
+    if scatter_fn is None:
+        from . import attn_fwd_jvp_scatter as scatter_fn
     # every rank has copied its previous results out of its slice buffer
     sb.barrier()
-    attn_fwd_jvp_scatter(*full.unbind(0), mask, sb.o, sb.to, sb.lse, sb.tlse, head_base=sb.rank * Hp,
-                         scale=scale, clean_tangent_zero=clean_tangent_zero)
+    scatter_fn(*full.unbind(0), mask, sb.o, sb.to, sb.lse, sb.tlse, head_base=sb.rank * Hp,
+               scale=scale, clean_tangent_zero=clean_tangent_zero)
     # every rank's rows have landed in this rank's slice buffer
     sb.barrier()
     me = sb.rank

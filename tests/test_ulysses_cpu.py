@@ -89,3 +89,82 @@ def test_single_rank_is_the_local_call():
     b = _oracle_local(*xs, mask)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+class _HostSlices:
+    """Slice buffers of the fused-output path for CPU ranks: shared-memory
+    tensors that every rank maps (entry r is rank r's slice), and a gloo barrier
+    in place of the stream-ordered one."""
+
+    def __init__(self, rank, o, to, lse, tlse):
+        self.rank = rank
+        self.o, self.to, self.lse, self.tlse = o, to, lse, tlse
+
+    def barrier(self):
+        dist.barrier()
+
+
+def _oracle_scatter(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, head_base, scale=None,
+                    clean_tangent_zero=False):
+    """What the scattering kernel does, with the oracle as the arithmetic: this
+    rank's heads over the whole sequence, each row stored into the slice that
+    owns its token, at the rank's head offset."""
+    ro, rto, rlse, rtlse = _oracle_local(q, k, v, tq, tk, tv, mask, scale=scale)
+    P, Hp = len(o), q.shape[1]
+    Ls = q.shape[2] // P
+    hs = slice(head_base, head_base + Hp)
+    for r in range(P):
+        rows = slice(r * Ls, (r + 1) * Ls)
+        o[r][:, hs] = ro[:, :, rows]
+        to[r][:, hs] = rto[:, :, rows]
+        lse[r][:, hs] = rlse[:, :, rows]
+        tlse[r][:, hs] = rtlse[:, :, rows]
+
+
+def _fused_worker(rank, world, port, mask, B, H, D, slices, q_out):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from masked_attention_jvp_b200.ulysses import _ulysses_fused_output
+        Ls = mask.seq_len // world
+        sb = _HostSlices(rank, *slices)
+        outs = []
+        for seed in (11, 12):  # the second call reuses the slice buffers
+            full = _inputs(B, H, mask.seq_len, D, seed=seed)
+            shard = torch.stack([x[:, :, rank * Ls:(rank + 1) * Ls].contiguous() for x in full])
+            res = _ulysses_fused_output(shard, mask, None, None, False, slices=sb, scatter_fn=_oracle_scatter)
+            outs.append([t.numpy() for t in res])
+        q_out.put((rank, outs))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,mask", [(2, MaskDesc(3, 1, 4, 1)), (4, MaskDesc(2, 2, 4, 1))])
+def test_fused_output_control_flow_matches_unsharded_oracle(world, mask):
+    """The fused-output path at world sizes 2 and 4: input all-to-all, each
+    rank's head offset, both barriers and the copy-out, twice over the same
+    slice buffers, against the oracle on the unsharded problem."""
+    import oracle
+    B, H, D = 1, 4, 8
+    Ls = mask.seq_len // world
+    nan = float("nan")
+    slices = tuple([torch.full(shape, nan, dtype=torch.float64).share_memory_() for _ in range(world)]
+                   for shape in ((B, H, Ls, D), (B, H, Ls, D), (B, H, Ls), (B, H, Ls)))
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_fused_worker, args=(r, world, port, mask, B, H, D, slices, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for call, seed in enumerate((11, 12)):
+        want = oracle.attn_fwd_jvp(*_inputs(B, H, mask.seq_len, D, seed=seed), mask)
+        for r in range(world):
+            sl = slice(r * Ls, (r + 1) * Ls)
+            for x, y in zip(got[r][call], want):
+                assert np.array_equal(x, y[:, :, sl]), (r, call)
