@@ -45,8 +45,8 @@ BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct 
 MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "89634e6b4f35b9e7"): 1431131648 + 390999296}
 PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241276160 + 1150380544}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
-BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "97e98721674f6154"):
-                    402571008 + 5875712 + 813365248 + 184498432 + 815200768 + 383543296}
+BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "74e781d6a3434c53"):
+                    402579712 + 8373760 + 814591488 + 183904256 + 817019904 + 383885056}
 
 
 def kernel_sources_hash(files=KERNEL_SOURCES) -> str:

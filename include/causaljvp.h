@@ -288,8 +288,10 @@ uint32_t caj_last_device_error_code(void);
 caj_status caj_set_wait_timeout_ms(double ms);
 
 /* Test hook for the bounded-wait path: mode 1 makes later tensor-core launches
- * skip the query-tile copies, so the MMA warp's first wait runs out, the kernel
- * records CAJ_ERR_DEVICE_TIMEOUT (site 3) and every role exits cleanly. Nothing
+ * skip their copies (the forward kernels: the query-tile copies; the backward's
+ * dQ and dK/dV kernels: every copy), so the MMA warp's first wait runs out, the
+ * kernel records CAJ_ERR_DEVICE_TIMEOUT with the site of that wait and every
+ * role exits cleanly. Nothing is in flight when the roles exit, and nothing
  * faults or hangs; outputs of such a call are undefined. mode 0 (default)
  * restores normal operation. Returns CAJ_OK, or CAJ_ERR_INVALID_ARG. */
 caj_status caj_debug_set_fault(int32_t mode);

@@ -671,6 +671,7 @@ caj_status caj_attn_bwd(const void *q, const void *k, const void *v, const void 
   p.n_row_tiles = ntile;
   p.scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt(float(D));
   p.timeout_ns = wait_timeout_ns();
+  p.fault_mode = g_fault_mode.load();
   // Launch orders: query tiles by decreasing key-tile count, key tiles by
   // decreasing query-tile count (ties: later first).
   std::vector<std::pair<int32_t, int32_t>> cq(ntile), ck(ntile);

@@ -267,25 +267,29 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    const uint32_t leader = elect_one();
-    int32_t armed = 0;
-    for (int32_t j = 0; j < ntiles; ++j) {
-      const int s = j % C::STAGES;
-      if (j >= C::STAGES && !bwarp_wait(bar.st_empty + 8 * s, ((j / C::STAGES) - 1) & 1, abort_flag,
-                                        p.timeout_ns, 21))
-        break;
-      const int32_t key0 = nth_tile(j, t) * BN;
-      const uint32_t dst = sbase + C::OFF_ST + s * C::STAGE, fb = bar.st_full + 8 * s;
-      mbar_arrive_expect_tx_if(leader, fb, 2 * C::S_BYTES);
+    // (test hook, fault_mode 1: no copies at all, so the MMA warp's first
+    // bounded wait runs out with nothing in flight)
+    if (p.fault_mode != 1) {
+      const uint32_t leader = elect_one();
+      int32_t armed = 0;
+      for (int32_t j = 0; j < ntiles; ++j) {
+        const int s = j % C::STAGES;
+        if (j >= C::STAGES && !bwarp_wait(bar.st_empty + 8 * s, ((j / C::STAGES) - 1) & 1, abort_flag,
+                                          p.timeout_ns, 21))
+          break;
+        const int32_t key0 = nth_tile(j, t) * BN;
+        const uint32_t dst = sbase + C::OFF_ST + s * C::STAGE, fb = bar.st_full + 8 * s;
+        mbar_arrive_expect_tx_if(leader, fb, 2 * C::S_BYTES);
 #pragma unroll
-      for (int c = 0; c < C::NB; ++c) {
-        tma_load_3d(leader, dst + c * C::SBLK, &p.tm_k_s, fb, c * 64, key0, bh);
-        tma_load_3d(leader, dst + C::S_BYTES + c * C::SBLK, &p.tm_v_s, fb, c * 64, key0, bh);
+        for (int c = 0; c < C::NB; ++c) {
+          tma_load_3d(leader, dst + c * C::SBLK, &p.tm_k_s, fb, c * 64, key0, bh);
+          tma_load_3d(leader, dst + C::S_BYTES + c * C::SBLK, &p.tm_v_s, fb, c * 64, key0, bh);
+        }
+        armed = j + 1;
       }
-      armed = j + 1;
+      for (int32_t j = (armed > C::STAGES ? armed - C::STAGES : 0); j < armed; ++j)
+        bdrain(bar.st_full + 8 * (j % C::STAGES), (j / C::STAGES) & 1, p.timeout_ns);
     }
-    for (int32_t j = (armed > C::STAGES ? armed - C::STAGES : 0); j < armed; ++j)
-      bdrain(bar.st_full + 8 * (j % C::STAGES), (j / C::STAGES) & 1, p.timeout_ns);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     const uint32_t leader = elect_one();
@@ -454,40 +458,44 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    const uint32_t leader = elect_one();
-    mbar_arrive_expect_tx_if(leader, bar.r_full, C::R_BYTES);
-    for (int c = 0; c < C::NB; ++c)
-      tma_load_3d(leader, sbase + C::OFF_R + c * C::RBLK, &p.tm_v_r, bar.r_full, c * 64, k0, bh);
-    int32_t armed = 0;
-    for (int32_t j = 0; j < ntiles; ++j) {
-      const int s = j % C::STAGES;
-      if (j >= C::STAGES && !bwarp_wait(bar.st_empty + 8 * s, ((j / C::STAGES) - 1) & 1, abort_flag,
-                                        p.timeout_ns, 31))
-        break;
-      const int32_t qb = nth_tile(j, t) * BN;
-      const uint32_t dst = sbase + C::OFF_ST + s * C::STAGE, fb = bar.st_full + 8 * s;
-      // row statistics of the 64 queries (LSE in base 2, Delta), +inf / 0 past N
-      float *stat = reinterpret_cast<float *>(sgen + C::OFF_ST + s * C::STAGE + 2 * C::S_BYTES);
+    // (test hook, fault_mode 1: no copies at all, so the MMA warp's first
+    // bounded wait runs out with nothing in flight)
+    if (p.fault_mode != 1) {
+      const uint32_t leader = elect_one();
+      mbar_arrive_expect_tx_if(leader, bar.r_full, C::R_BYTES);
+      for (int c = 0; c < C::NB; ++c)
+        tma_load_3d(leader, sbase + C::OFF_R + c * C::RBLK, &p.tm_v_r, bar.r_full, c * 64, k0, bh);
+      int32_t armed = 0;
+      for (int32_t j = 0; j < ntiles; ++j) {
+        const int s = j % C::STAGES;
+        if (j >= C::STAGES && !bwarp_wait(bar.st_empty + 8 * s, ((j / C::STAGES) - 1) & 1, abort_flag,
+                                          p.timeout_ns, 31))
+          break;
+        const int32_t qb = nth_tile(j, t) * BN;
+        const uint32_t dst = sbase + C::OFF_ST + s * C::STAGE, fb = bar.st_full + 8 * s;
+        // row statistics of the 64 queries (LSE in base 2, Delta), +inf / 0 past N
+        float *stat = reinterpret_cast<float *>(sgen + C::OFF_ST + s * C::STAGE + 2 * C::S_BYTES);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int32_t qi = qb + 32 * h + lane;
-        const bool in = qi < p.geom.N;
-        const size_t idx = size_t(bh) * p.geom.N + (in ? qi : 0);
-        stat[32 * h + lane] = in ? p.lse[idx] * kLog2e : INFINITY;
-        stat[64 + 32 * h + lane] = in ? p.delta[idx] : 0.f;
-      }
-      __syncwarp();
-      mbar_arrive_expect_tx_if(leader, fb, 2 * C::S_BYTES);
+        for (int h = 0; h < 2; ++h) {
+          const int32_t qi = qb + 32 * h + lane;
+          const bool in = qi < p.geom.N;
+          const size_t idx = size_t(bh) * p.geom.N + (in ? qi : 0);
+          stat[32 * h + lane] = in ? p.lse[idx] * kLog2e : INFINITY;
+          stat[64 + 32 * h + lane] = in ? p.delta[idx] : 0.f;
+        }
+        __syncwarp();
+        mbar_arrive_expect_tx_if(leader, fb, 2 * C::S_BYTES);
 #pragma unroll
-      for (int c = 0; c < C::NB; ++c) {
-        tma_load_3d(leader, dst + c * C::SBLK, &p.tm_q_s, fb, c * 64, qb, bh);
-        tma_load_3d(leader, dst + C::S_BYTES + c * C::SBLK, &p.tm_do_s, fb, c * 64, qb, bh);
+        for (int c = 0; c < C::NB; ++c) {
+          tma_load_3d(leader, dst + c * C::SBLK, &p.tm_q_s, fb, c * 64, qb, bh);
+          tma_load_3d(leader, dst + C::S_BYTES + c * C::SBLK, &p.tm_do_s, fb, c * 64, qb, bh);
+        }
+        armed = j + 1;
       }
-      armed = j + 1;
+      bdrain(bar.r_full, 0, p.timeout_ns);
+      for (int32_t j = (armed > C::STAGES ? armed - C::STAGES : 0); j < armed; ++j)
+        bdrain(bar.st_full + 8 * (j % C::STAGES), (j / C::STAGES) & 1, p.timeout_ns);
     }
-    bdrain(bar.r_full, 0, p.timeout_ns);
-    for (int32_t j = (armed > C::STAGES ? armed - C::STAGES : 0); j < armed; ++j)
-      bdrain(bar.st_full + 8 * (j % C::STAGES), (j / C::STAGES) & 1, p.timeout_ns);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     const uint32_t leader = elect_one();

@@ -137,6 +137,7 @@ struct BwdParams {
   uint64_t timeout_ns;
   uint16_t row_order[kMaxQTiles];  // query tiles, heaviest first (dq kernel)
   uint16_t col_order[kMaxQTiles];  // key tiles, heaviest first (dkdv kernel)
+  int32_t fault_mode;     // test hook: 1 = the producers issue no copies
 };
 
 // Each returns the launch's cudaError_t (cudaSuccess when enqueued).

@@ -1,8 +1,9 @@
-"""Failure detection on the GPU without a fault: the tensor-core kernel's waits
-are bounded. With the library's test hook the query-tile copies are skipped, so
-the MMA warp's first wait can never complete; the kernel must give up after the
-configured limit, report CAJ_ERR_DEVICE_TIMEOUT through the device error word,
-leave the context usable, and the next normal call must be correct."""
+"""Failure detection on the GPU without a fault: the tensor-core kernels' waits
+are bounded. With the library's test hook the producers skip their copies (the
+forward's query tiles, every copy of the backward's), so the MMA warp's first
+wait can never complete; the kernel must give up after the configured limit,
+report CAJ_ERR_DEVICE_TIMEOUT through the device error word, leave the context
+usable, and the next normal call must be correct."""
 import numpy as np
 import pytest
 import torch
@@ -74,3 +75,36 @@ def test_clean_tangent_zero_kernels_time_out_too():
     rel = lambda a, b: float(np.linalg.norm(a - b) / np.linalg.norm(b))
     assert rel(o.float().cpu().numpy(), ro) <= 1e-2
     assert rel(to.float().cpu().numpy(), rto) <= 1e-2
+
+
+def test_backward_kernels_time_out_too():
+    """The backward's dQ and dK/dV kernels bound their waits the same way: with
+    the hook their producers issue no copies, the MMA warp's first wait runs
+    out, and the next normal call is correct."""
+    L = _lib.lib()
+    w = Workload("fault_bwd", 1, 1, 128, MaskDesc(64, 1, 2, 0), torch.bfloat16, seed=7)  # one tile each
+    q, k, v, _, _, _ = make_inputs(w, "cuda")
+    g = torch.Generator(device="cpu").manual_seed(8)
+    dout = torch.randn(q.shape, generator=g).to(torch.bfloat16).cuda()
+    z = torch.zeros_like(q)
+    o, _, lse, _ = caj.attn_fwd_jvp(q, k, v, z, z, z, w.mask)
+    caj.device_status()
+    assert L.caj_set_wait_timeout_ms(100.0) == _lib.CAJ_OK
+    assert L.caj_debug_set_fault(1) == _lib.CAJ_OK
+    try:
+        caj.attn_bwd(q, k, v, o, dout, lse, w.mask)
+        with pytest.raises(caj.CajError) as err:
+            caj.device_status()
+        assert err.value.status == _lib.CAJ_ERR_DEVICE_TIMEOUT
+        assert L.caj_last_device_error_code() & 0xFF00 == 0x100
+    finally:
+        L.caj_debug_set_fault(0)
+        L.caj_set_wait_timeout_ms(0.0)
+    caj.device_status()
+    dq, dk, dv, delta = caj.attn_bwd(q, k, v, o, dout, lse, w.mask)
+    caj.device_status()
+    rq, rk, rv, rdelta = oracle.attn_bwd(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), w.mask)
+    rel = lambda a, b: float(np.linalg.norm(a - b) / np.linalg.norm(b))
+    assert rel(dq.float().cpu().numpy(), rq) <= 2e-2
+    assert rel(dk.float().cpu().numpy(), rk) <= 2e-2
+    assert rel(dv.float().cpu().numpy(), rv) <= 1e-2
