@@ -89,3 +89,28 @@ def test_scatter_rejects_bad_slices():
     o, to, lse, tlse = _slices(1, 2, 32, 64, bf, 2, False)
     with pytest.raises(caj.CajError):  # heads 1, 2 of a 2-head slice
         caj.attn_fwd_jvp_scatter(*ins, w.mask, o, to, lse, tlse, head_base=1)
+
+
+def test_scatter_at_full_size_equals_direct_call():
+    """The bench's scatter configuration at full size: the TF frame-wise
+    workload (B=1, H=12, N=65520, D=128) split over 4 emulated ranks of 3 heads,
+    slices of 16380 rows (query tiles straddle every slice boundary)."""
+    from masked_attention_jvp_b200.workloads import WORKLOADS
+    w = WORKLOADS["wan1.3b_tf_framewise"]
+    P = 4
+    ins = make_inputs(w, "cuda")
+    direct = caj.attn_fwd_jvp(*ins, w.mask)
+    Hp, Ls = w.H // P, w.N // P
+    o, to, lse, tlse = _slices(w.B, w.H, Ls, w.D, w.dtype, P, False)
+    for r in range(P):
+        mine = [x[:, r * Hp:(r + 1) * Hp].contiguous() for x in ins]
+        caj.attn_fwd_jvp_scatter(*mine, w.mask, o, to, lse, tlse, head_base=r * Hp)
+        del mine
+    torch.cuda.synchronize()
+    caj.device_status()
+    for r in range(P):
+        rows = slice(r * Ls, (r + 1) * Ls)
+        assert torch.equal(o[r], direct[0][:, :, rows])
+        assert torch.equal(to[r], direct[1][:, :, rows])
+        assert torch.equal(lse[r], direct[2][:, :, rows])
+        assert torch.equal(tlse[r], direct[3][:, :, rows])
