@@ -41,27 +41,41 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct Sm100Params"]
 PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
 BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
-# {(workload, sources_sha256): dram bytes read + written per launch}
-MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "89634e6b4f35b9e7"): 1431131648 + 390999296}
-PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "ac05fd3e4a3bd17a"): 1241276160 + 1150380544}
+# {(workload, code hash of the kernel's sources): dram bytes read + written per launch}
+MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "2eecf04220eab7c1"): 1431131648 + 390999296}
+PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "34494554b0571872"): 1241276160 + 1150380544}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
-BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "74e781d6a3434c53"):
+BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "eb90badc0d3e064a"):
                     402579712 + 8373760 + 814591488 + 183904256 + 817019904 + 383885056}
 
 
-def kernel_sources_hash(files=KERNEL_SOURCES) -> str:
+def _code_only(text: str) -> str:
+    """The code of a C/CUDA source: comments removed, whitespace runs collapsed,
+    so that editing a comment does not invalidate measured counters."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_sources_hash(files=KERNEL_SOURCES, read=None) -> str:
+    """sha256 prefix over the code (not the comments) of a kernel's sources and
+    its parameter struct. `read(name)` returns a file of csrc/ as text (default:
+    the working tree)."""
     import hashlib
     import re
     csrc = os.path.join(ROOT, "masked_attention_jvp_b200", "csrc")
+    if read is None:
+        def read(name):
+            with open(os.path.join(csrc, name), encoding="utf-8") as fh:
+                return fh.read()
     h = hashlib.sha256()
     for f in files:
         if f.startswith("struct "):
-            text = open(os.path.join(csrc, "kernels.h")).read()
-            m = re.search(r"^%s \{.*?^\};" % re.escape(f), text, re.S | re.M)
-            h.update(m.group(0).encode() if m else f.encode())
+            m = re.search(r"^%s \{.*?^\};" % re.escape(f), read("kernels.h"), re.S | re.M)
+            h.update(_code_only(m.group(0) if m else f).encode())
         else:
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+            h.update(_code_only(read(f)).encode())
     return h.hexdigest()[:16]
 
 

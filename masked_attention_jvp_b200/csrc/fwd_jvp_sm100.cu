@@ -194,17 +194,10 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, timeout_ns, site));
 }
 
-// KIND (a TileKind): dense tangents (kTilesAll), or the query tiles with a noisy
-// row under clean-tangent-zero teacher forcing (kTilesNoisyCTZ: the caller
-// guarantees tq, tk, tv vanish on rows < L). Each is its own instantiation, so
-// the dense kernel carries no trace of the specialisation; the clean query
-// tiles have a kernel of their own (fwd_primal_sm100_kernel). Measured on the
-// TF frame-wise workload: one kernel branching on the kind of each tile took
-// 16.0 ms, the two specialised launches 12.0 ms.
 // The slice-map arithmetic of the scattering epilogues, kept out of line.
 // Inlined, it changed the register allocation of the kernels' main loop:
 // the scattering kernel then ran 4.7% slower than the plain one, against
-// 2.9% out of line (3 heads of the TF frame-wise workload, round-robin).
+// 2.5-2.9% out of line (3 heads of the TF frame-wise workload, round-robin).
 __device__ __noinline__ void scatter_rows(const OutMap &m, int32_t bh, int32_t q, int D, uint4 **o,
                                           uint4 **to) {
   const OutRow dst = slice_row(m, bh, q);
@@ -218,6 +211,17 @@ __device__ __noinline__ void scatter_stats(const OutMap &m, int32_t bh, int32_t 
   m.tlse[dst.shard][dst.stat] = tlse;
 }
 
+// KIND (a TileKind): dense tangents (kTilesAll), or the query tiles with a noisy
+// row under clean-tangent-zero teacher forcing (kTilesNoisyCTZ: the caller
+// guarantees tq, tk, tv vanish on rows < L). Each is its own instantiation, so
+// the dense kernel carries no trace of the specialisation; the clean query
+// tiles have a kernel of their own (fwd_primal_sm100_kernel). Measured on the
+// TF frame-wise workload: one kernel branching on the kind of each tile took
+// 16.0 ms, the two specialised launches 12.0 ms.
+// SCATTER: the epilogue stores each row into its sequence slice through the
+// slice map (caj_attn_fwd_jvp_scatter, the Ulysses output all-to-all) instead
+// of the one-slice output; a separate instantiation, so the one-slice kernel
+// keeps its plain addressing.
 template <int D, int KIND, bool SCATTER>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_jvp_sm100_kernel(const __grid_constant__ Sm100Params p) {

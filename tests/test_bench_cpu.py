@@ -40,3 +40,20 @@ def test_warmup_below_three_is_refused():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"], capture_output=True,
                        text=True, timeout=120, cwd=ROOT)
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_traffic_key_ignores_comments_but_not_code():
+    """The DRAM-traffic tables are keyed by a hash of the kernel's code: a
+    comment edit keeps the key, a code edit changes it."""
+    import bench
+    src = {"a.cu": "int f(int x) { // double it\n  return 2 * x; /* twice */ }\n",
+           "kernels.h": "struct P {\n  int n;  // rows\n};\n"}
+    files = ["a.cu", "struct P"]
+    base = bench.kernel_sources_hash(files, src.get)
+    recommented = {"a.cu": "// doubles its argument\nint f(int x) {\n  return 2 * x;\n}\n",
+                   "kernels.h": "struct P {\n  int n;\n};\n"}
+    assert bench.kernel_sources_hash(files, recommented.get) == base
+    changed = dict(src, **{"a.cu": src["a.cu"].replace("2 * x", "3 * x")})
+    assert bench.kernel_sources_hash(files, changed.get) != base
+    changed = dict(src, **{"kernels.h": "struct P {\n  long n;\n};\n"})
+    assert bench.kernel_sources_hash(files, changed.get) != base
