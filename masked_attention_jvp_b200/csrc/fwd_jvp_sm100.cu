@@ -197,7 +197,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // The slice-map arithmetic of the scattering epilogues, kept out of line.
 // Inlined, it changed the register allocation of the kernels' main loop:
 // the scattering kernel then ran 4.7% slower than the plain one, against
-// 2.5-2.9% out of line (3 heads of the TF frame-wise workload, round-robin).
+// 2.5-4.2% out of line (3 heads of the TF frame-wise workload, round-robin).
 __device__ __noinline__ void scatter_rows(const OutMap &m, int32_t bh, int32_t q, int D, uint4 **o,
                                           uint4 **to) {
   const OutRow dst = slice_row(m, bh, q);
