@@ -102,14 +102,33 @@ class SliceBuffers:
         self.handle.barrier(channel=0, timeout_ms=timeout_ms)
 
 
+class _LocalSlices:
+    """The one slice of a single process without a process group: ordinary
+    device memory, and nothing to wait for."""
+
+    def __init__(self, B: int, H: int, Ls: int, D: int, dtype: torch.dtype, device):
+        self.rank, self.world = 0, 1
+        self.o = [torch.empty(B, H, Ls, D, dtype=dtype, device=device)]
+        self.to = [torch.empty_like(self.o[0])]
+        self.lse = [torch.empty(B, H, Ls, dtype=torch.float32, device=device)]
+        self.tlse = [torch.empty_like(self.lse[0])]
+
+    def barrier(self, timeout_ms: int = 10000):
+        pass
+
+
 _slice_buffers = {}
 
 
-def _get_slice_buffers(B, H, Ls, D, dtype, device, group) -> SliceBuffers:
+def _get_slice_buffers(B, H, Ls, D, dtype, device, group):
     key = (B, H, Ls, D, dtype, torch.device(device), id(group))
     sb = _slice_buffers.get(key)
     if sb is None:
-        sb = _slice_buffers[key] = SliceBuffers(B, H, Ls, D, dtype, device, group)
+        if dist.is_initialized():
+            sb = SliceBuffers(B, H, Ls, D, dtype, device, group)
+        else:
+            sb = _LocalSlices(B, H, Ls, D, dtype, device)
+        _slice_buffers[key] = sb
     return sb
 
 
@@ -129,7 +148,8 @@ def ulysses_attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = Non
     is done by the kernel's epilogue, which stores each row into the
     symmetric-memory slice buffer of its owner (see SliceBuffers). The
     returned tensors are copies, so the slice buffers are free for the next
-    call once every rank has passed its first barrier.
+    call once every rank has passed its first barrier. Without a process group
+    (a single process) the one slice is ordinary device memory.
     """
     ins = torch.stack([q, k, v, tq, tk, tv])
     if fused_output:

@@ -168,3 +168,20 @@ def test_fused_output_control_flow_matches_unsharded_oracle(world, mask):
             sl = slice(r * Ls, (r + 1) * Ls)
             for x, y in zip(got[r][call], want):
                 assert np.array_equal(x, y[:, :, sl]), (r, call)
+
+
+def test_fused_output_without_process_group_is_the_local_call():
+    """A single process with no process group: the fused path uses one local
+    slice and no barrier, and returns the local attention."""
+    from masked_attention_jvp_b200.ulysses import _ulysses_fused_output, release_slice_buffers
+    assert not dist.is_initialized()
+    mask = MaskDesc(3, 1, 3, 1)
+    xs = _inputs(1, 2, mask.seq_len, 4, seed=5)
+    try:
+        got = _ulysses_fused_output(torch.stack(xs), mask, None, None, False, scatter_fn=_oracle_scatter)
+    finally:
+        release_slice_buffers()
+    o, to, lse, tlse = _oracle_local(*xs, mask)
+    assert torch.equal(got[0], o) and torch.equal(got[1], to)
+    # the statistics slices are fp32, as the kernel writes them
+    assert torch.equal(got[2], lse.float()) and torch.equal(got[3], tlse.float())
