@@ -50,6 +50,9 @@ def _load():
         lib.oracle_qk_norm_rope_jvp.restype = i32
         lib.oracle_attn_bwd.argtypes = [vp] * 4 + [i32, i64, i64, i64, dbl, i64, i64, i64, i32] + [vp] * 4
         lib.oracle_attn_bwd.restype = i32
+        lib.oracle_attn_bwd_dq_rows.argtypes = [vp] * 4 + [i32, i64, i64, i64, dbl, i64, i64, i64, i32,
+                                                           vp, i64, vp, vp]
+        lib.oracle_attn_bwd_dq_rows.restype = i32
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i32
         _lib = lib
@@ -180,6 +183,31 @@ def attn_bwd(q, k, v, dout, mask, scale=None):
     if rc != 0:
         raise ValueError("oracle: rejected arguments")
     return dq, dk, dv, delta
+
+
+def attn_bwd_dq_rows(q, k, v, dout, mask, rows, scale=None):
+    """fp64 dQ and Delta of selected query rows (flat ids bh*N + i) of the
+    masked attention backward. Each row needs only its own softmax, so this
+    serves full-size problems where the N x N backward would not finish.
+    Returns numpy arrays dq [R, D] and delta [R] (float64)."""
+    ts = [_as_host(t) for t in (q, k, v, dout)]
+    dtypes = {d for _, d in ts}
+    if len(dtypes) != 1:
+        raise TypeError("oracle: all four inputs must share one dtype")
+    dtype = dtypes.pop()
+    B, H, N, D = q.shape
+    T, c, F, tf = _mask_tuple(mask)
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(D))
+    rows = torch.as_tensor(rows, dtype=torch.int64).contiguous()
+    R = rows.numel()
+    dq = np.zeros((R, D), np.float64)
+    delta = np.zeros((R,), np.float64)
+    rc = _load().oracle_attn_bwd_dq_rows(*[t.data_ptr() for t, _ in ts], dtype, B * H, N, D, float(scale),
+                                         T, c, F, tf, rows.data_ptr(), R, dq.ctypes.data, delta.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle: rejected arguments")
+    return dq, delta
 
 
 def out_proj_jvp(x, tx, w, bias=None):

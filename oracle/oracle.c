@@ -347,3 +347,79 @@ int oracle_attn_bwd(const void *q, const void *k, const void *v, const void *dou
   }
   return bad ? -1 : 0;
 }
+
+/*
+ * dQ and Delta of selected query rows (the same definitions as oracle_attn_bwd,
+ * restricted to rows). Row i needs only its own softmax:
+ *   p_j = exp(s_j - m) / Z over the keys row i sees,  dp_j = <dO_i, v_j>,
+ *   Delta_i = sum_j p_j dp_j,  dQ_i = scale sum_j p_j (dp_j - Delta_i) k_j.
+ * So a few hundred rows of a full-size problem cost a few hundred row passes,
+ * not the whole N x N backward.
+ *   q, k, v, dout : [BH, N, D] in `dtype`;  rows : flat ids bh*N + i
+ *   dq            : [nrows, D] double;  delta : [nrows] double
+ */
+int oracle_attn_bwd_dq_rows(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                            int64_t BH, int64_t N, int64_t D, double scale, int64_t T, int64_t c,
+                            int64_t F, int tf, const int64_t *rows, int64_t nrows, double *dq,
+                            double *delta) {
+  if (D <= 0 || N <= 0 || BH <= 0 || nrows < 0) return -1;
+  if (N != F * T * (tf ? 2 : 1)) return -1;
+  for (int64_t r = 0; r < nrows; ++r)
+    if (rows[r] < 0 || rows[r] >= BH * N) return -1;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+    int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+    if (!p || !dp || !keys) {
+#pragma omp atomic write
+      bad = 1;
+    } else {
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t bh = rows[r] / N, i = rows[r] % N, head = bh * N * D;
+        double *dqrow = dq + r * D;
+        for (int64_t d = 0; d < D; ++d) dqrow[d] = 0.0;
+        int64_t nk = 0;
+        for (int64_t j = 0; j < N; ++j)
+          if (oracle_visible(T, c, F, tf, i, j)) keys[nk++] = j;
+        if (nk == 0) {
+          delta[r] = 0.0;
+          continue;
+        }
+        double m = -INFINITY;
+        for (int64_t a = 0; a < nk; ++a) {
+          double s = 0.0, t = 0.0;
+          for (int64_t d = 0; d < D; ++d) {
+            s += load_elem(q, dtype, head + i * D + d) * load_elem(k, dtype, head + keys[a] * D + d);
+            t += load_elem(dout, dtype, head + i * D + d) * load_elem(v, dtype, head + keys[a] * D + d);
+          }
+          p[a] = scale * s;
+          dp[a] = t;
+          if (p[a] > m) m = p[a];
+        }
+        double Z = 0.0;
+        for (int64_t a = 0; a < nk; ++a) {
+          p[a] = exp(p[a] - m);
+          Z += p[a];
+        }
+        double dl = 0.0;
+        for (int64_t a = 0; a < nk; ++a) {
+          p[a] /= Z;
+          dl += p[a] * dp[a];
+        }
+        delta[r] = dl;
+        for (int64_t a = 0; a < nk; ++a) {
+          const double ds = p[a] * (dp[a] - dl);
+          for (int64_t d = 0; d < D; ++d)
+            dqrow[d] += scale * ds * load_elem(k, dtype, head + keys[a] * D + d);
+        }
+      }
+    }
+    free(p);
+    free(dp);
+    free(keys);
+  }
+  return bad ? -1 : 0;
+}

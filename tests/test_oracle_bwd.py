@@ -86,3 +86,43 @@ def test_single_key_row_has_no_query_gradient():
     q, k, v, dout = rand(1, 1, mask.seq_len, 4, seed=7)
     dq, _, _, _ = oracle.attn_bwd(q, k, v, dout, mask)
     assert np.all(dq[0, 0, 0] == 0.0)
+
+
+@pytest.mark.parametrize("mask", MASKS)
+def test_dq_rows_match_central_differences_of_the_forward(mask):
+    """dQ of one row from the row-wise oracle equals the central difference of
+    <dO, O> when only that row of q moves (the forward oracle, h = 1e-6)."""
+    q, k, v, dout = rand(1, 2, mask.seq_len, 6, seed=8)
+    (u,) = rand(1, 2, mask.seq_len, 6, seed=9, n=1)
+    N = mask.seq_len
+    for bh, i in ((0, 0), (1, N - 1), (0, N // 2)):
+        e = torch.zeros_like(u)
+        e[0, bh, i] = u[0, bh, i]
+        dq, _ = oracle.attn_bwd_dq_rows(q, k, v, dout, mask, rows=[bh * N + i])
+        h = 1e-6
+        fd = (loss(q + h * e, k, v, dout, mask) - loss(q - h * e, k, v, dout, mask)) / (2 * h)
+        an = float(np.sum(dq[0] * u[0, bh, i].numpy()))
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (bh, i, fd, an)
+
+
+@pytest.mark.parametrize("mask", MASKS)
+def test_dq_rows_delta_is_the_output_inner_product(mask):
+    """Delta_i = <dO_i, O_i>, with O from the forward oracle; every row's dQ
+    also equals that row of the full backward."""
+    q, k, v, dout = rand(2, 2, mask.seq_len, 5, seed=10)
+    N = mask.seq_len
+    rows = torch.arange(4 * N)
+    dq, delta = oracle.attn_bwd_dq_rows(q, k, v, dout, mask, rows=rows)
+    z = torch.zeros_like(q)
+    o, _, _, _ = oracle.attn_fwd_jvp(q, k, v, z, z, z, mask)
+    assert np.max(np.abs(delta - np.sum(o * dout.numpy(), axis=-1).reshape(-1))) <= 1e-12
+    fdq, _, _, _ = oracle.attn_bwd(q, k, v, dout, mask)
+    assert np.max(np.abs(dq - fdq.reshape(-1, 5))) <= 1e-12
+
+
+def test_dq_rows_single_key_row_is_zero():
+    mask = MaskDesc(1, 1, 4, 0)
+    q, k, v, dout = rand(1, 1, mask.seq_len, 4, seed=11)
+    dq, delta = oracle.attn_bwd_dq_rows(q, k, v, dout, mask, rows=[0])
+    assert np.all(dq == 0.0)
+    assert abs(delta[0] - float(dout[0, 0, 0] @ v[0, 0, 0])) <= 1e-12
