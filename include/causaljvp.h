@@ -195,6 +195,39 @@ caj_status caj_attn_fwd_jvp_host(const void *q, const void *k, const void *v,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * caj_attn_fwd_jvp_host with no device memory from the caller. The paper has
+ * no counterpart to this call; it exists for callers that cannot allocate
+ * device memory: a plain C program or plugin that keeps its tensors in host
+ * memory and links no device allocator, or a host runtime whose memory manager
+ * owns every device allocation and forbids cudaMalloc from its extensions.
+ * The device staging area is a fixed array of CAJ_HOST_STATIC_MAX_BYTES inside
+ * the library (a file-scope __device__ array). Every device that loads the
+ * library holds it until the process exits. Nothing is allocated or freed by
+ * the call: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   in / out       as caj_attn_fwd_jvp_host (host buffers; pinned memory lets
+ *                  the copies overlap the kernels)
+ *   size limit     the problem's caj_attn_fwd_jvp_host_workspace() size must
+ *                  not exceed CAJ_HOST_STATIC_MAX_BYTES (for bf16, D = 128:
+ *                  B*H*N up to about 32 000 rows). A larger problem returns
+ *                  CAJ_ERR_UNSUPPORTED and touches nothing.
+ *   first call     the first call on each device looks up the array's device
+ *                  address (cudaGetSymbolAddress, with that device current).
+ *                  Make that first call before any stream capture.
+ *   sharing        every call on a device uses the same array, which keeps the
+ *                  last call's contents. Each call overwrites every byte it
+ *                  reads back, so nothing needs clearing. Calls whose work
+ *                  overlaps on the GPU (other streams, other host threads)
+ *                  race on the array: order them, e.g. on one stream.
+ * Returns as caj_attn_fwd_jvp_host, CAJ_ERR_UNSUPPORTED for a problem beyond
+ * the limit, or CAJ_ERR_CUDA if the array's address cannot be looked up.
+ */
+#define CAJ_HOST_STATIC_MAX_BYTES (64u << 20)
+caj_status caj_attn_fwd_jvp_host_static(const void *q, const void *k, const void *v,
+                                        const void *tq, const void *tk, const void *tv,
+                                        const caj_problem *prob, const caj_mask_desc *mask,
+                                        void *o, void *to, float *lse, float *tlse, void *stream);
+
+/*
  * Output projection of the attention block in primal-tangent form. Causal-rCM
  * runs the JVP layer by layer, each layer mapping a (primal, tangent) pair to a
  * pair (section 3.2.2, "JVP FSDP2"); the projection after attention is

@@ -28,7 +28,7 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -162,6 +162,42 @@ def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
                                  ctypes.c_void_p(workspace.data_ptr()), nbytes,
                                  ctypes.c_void_p(stream.cuda_stream))
     _lib.check(st, "caj_attn_fwd_jvp_host")
+    stream.synchronize()
+    return o, to, lse, tlse
+
+
+def attn_fwd_jvp_host_static(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,
+                             clean_tangent_zero: bool = False):
+    """Host tensors in, pinned host tensors out, with no device memory
+    allocated anywhere: the library stages the call in a fixed device array of
+    its own (caj_attn_fwd_jvp_host_static). This is for callers that cannot
+    allocate device memory, e.g. a host runtime whose allocator owns the GPU.
+    The problem's staging must fit in HOST_STATIC_MAX_BYTES (64 MiB); calls
+    share that array, so calls overlapping on the GPU race. The first call on
+    a device looks up the array's address: make it before any stream capture.
+    Returns (o, to, lse, tlse) like attn_fwd_jvp on host tensors."""
+    ins = (q, k, v, tq, tk, tv)
+    for t in ins:
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("attn_fwd_jvp_host_static: inputs must be contiguous CPU tensors")
+    if q.dtype not in _DTYPES or any(t.dtype != q.dtype or t.shape != q.shape for t in ins):
+        raise ValueError("attn_fwd_jvp_host_static: q..tv must share one shape and dtype (bf16 or fp32)")
+    prob = _problem(q, scale, clean_tangent_zero)
+    L = _lib.lib()
+    o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    to = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)
+    tlse = torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True)
+    stream = torch.cuda.current_stream(torch.device("cuda", torch.cuda.current_device()))
+    st = L.caj_attn_fwd_jvp_host_static(*[ctypes.c_void_p(t.data_ptr()) for t in ins], ctypes.byref(prob),
+                                        ctypes.byref(_lib.mask_c(mask)),
+                                        *[ctypes.c_void_p(t.data_ptr()) for t in (o, to, lse, tlse)],
+                                        ctypes.c_void_p(stream.cuda_stream))
+    if st == _lib.CAJ_ERR_UNSUPPORTED:
+        raise _lib.CajError(st, "caj_attn_fwd_jvp_host_static: the problem's staging exceeds the "
+                                f"library's fixed {_lib.HOST_STATIC_MAX_BYTES >> 20} MiB device array "
+                                "(or D is not 64/128)")
+    _lib.check(st, "caj_attn_fwd_jvp_host_static")
     stream.synchronize()
     return o, to, lse, tlse
 

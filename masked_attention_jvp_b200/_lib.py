@@ -18,11 +18,12 @@ EXPORTED = [
     "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
     "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
     "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host", "caj_out_proj_jvp",
-    "caj_attn_fwd_jvp_scatter",
+    "caj_attn_fwd_jvp_scatter", "caj_attn_fwd_jvp_host_static",
 ]
 
 
 MAX_SHARDS = 8  # CAJ_MAX_SHARDS
+HOST_STATIC_MAX_BYTES = 64 << 20  # CAJ_HOST_STATIC_MAX_BYTES
 
 
 class SeqScatterC(ctypes.Structure):
@@ -111,6 +112,9 @@ def lib() -> ctypes.CDLL:
         L.caj_attn_fwd_jvp_host.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC)] + \
             [vp] * 5 + [ctypes.c_size_t, vp]
         L.caj_attn_fwd_jvp_host.restype = ctypes.c_int
+        L.caj_attn_fwd_jvp_host_static.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC),
+                                                    ctypes.POINTER(MaskDescC)] + [vp] * 5
+        L.caj_attn_fwd_jvp_host_static.restype = ctypes.c_int
         L.caj_out_proj_jvp.argtypes = [vp] * 4 + [ctypes.POINTER(LinearShapeC), vp, vp, vp]
         L.caj_out_proj_jvp.restype = ctypes.c_int
         L.caj_attn_fwd_jvp_scatter.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC),
