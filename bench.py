@@ -3,13 +3,19 @@
 One step = one call of the fused kernel over the whole workload (every head of
 every batch entry), inputs resident in HBM. Default workload: the teacher-forcing
 frame-wise Wan2.1-1.3B-shaped layout (B=1, H=12, D=128, 21 clean + 21 noisy
-latent frames of 1560 tokens, N=65520, bf16 in / fp32 accumulate).
+latent frames of 1560 tokens, N=65520, bf16 in / fp32 accumulate). The default
+single-GPU run also times the other four workloads (one key each under
+"configs"), the backward, the prologue, the output projection, the
+clean-tangent-zero call and the context-parallel scatter.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--split heads|replicas|ulysses] [--fused-output]
 
-Prints one JSON line on rank 0. Multi-GPU runs (torchrun) give every rank its
-own copy of the workload (independent problems, no data-path collective) and
-report whole-job throughput over the slowest rank.
+Prints one JSON line on rank 0. Multi-GPU runs (torchrun) split one problem:
+by default its heads go to the ranks (independent problems, no data-path
+collective, strong scaling); --split ulysses gives every rank a sequence shard
+and runs the Ulysses all-to-all path; --split replicas gives every rank its own
+copy (weak scaling). Throughput is whole-job work over the slowest rank's time.
 """
 from __future__ import annotations
 
@@ -293,6 +299,22 @@ def whole_job_tflops(flops_per_rank: int, world: int, steps: int, slowest_ms: fl
     return world * flops_per_rank * steps / (slowest_ms / 1e3) / 1e12
 
 
+def split_heads(H: int, world: int, rank: int):
+    """Heads [h0, h1) of `rank` when one problem's H heads are spread over
+    `world` ranks as evenly as they go (the first H % world ranks take one
+    more). Heads are independent problems, so no collective joins them."""
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def strong_tflops(total_flops: int, steps: int, slowest_ms: float) -> float:
+    """Whole-job throughput of one problem split over the ranks (strong
+    scaling): the whole problem's work per step, done within the slowest
+    rank's time."""
+    return total_flops * steps / (slowest_ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------ prologue
 def bench_prologue(w, dev, steps, peaks):
     """The attention block's prologue in primal-tangent form (QK-RMSNorm + JVP,
@@ -479,29 +501,115 @@ def bench_cp_scatter(w, ins, steps, fl):
     return res
 
 
+# ------------------------------------------------------- the other workloads
+def bench_config(name, steps, warmup, peaks, with_cpu=True, cpu_target_s=5.0):
+    """One of the other workloads, timed like the headline: `warmup` calls,
+    then `steps` calls back to back with CUDA events, SM clocks sampled during
+    the loop. The bf16 workloads run the tensor-core kernel and carry a
+    roofline against the measured bf16 burst; the fp32 one runs the CUDA-core
+    kernel (one small launch, bound by launch latency). The oracle is timed on
+    a row sample of the same inputs beside it."""
+    import masked_attention_jvp_b200 as caj
+    w = WORKLOADS[name]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    host = make_inputs(w, "cpu")
+    ins = [t.to(dev) for t in host]
+    shape = ins[0].shape
+    o, to = torch.empty_like(ins[0]), torch.empty_like(ins[0])
+    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    tlse = torch.empty_like(lse)
+    fl = flops_of(w)
+
+    def step():
+        caj.attn_fwd_jvp_out(*ins, w.mask, o, to, lse, tlse, scale=w.scale)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    caj.device_status()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    with ClockSampler(dev.index) as clk:
+        ev[0].record()
+        for i in range(steps):
+            step()
+            ev[i + 1].record()
+        torch.cuda.synchronize()
+    caj.device_status()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    ms = statistics.mean(per)
+    tf = fl / (ms / 1e3) / 1e12
+    res = {"workload": name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "mask": list(w.mask.as_tuple()),
+           "dtype": "f32" if w.dtype == torch.float32 else "bf16",
+           "flop_per_call": fl, "ms_mean": round(ms, 4), "ms_median": round(statistics.median(per), 4),
+           "ms_min": round(min(per), 4), "tflops": round(tf, 3), "steps": steps, "warmup": warmup,
+           "clocks": clk.summary(), "gpu_launches": steps}
+    if w.dtype == torch.bfloat16:
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        res["kernel"] = "fwd_jvp_sm100_kernel<%d>" % w.D
+        res["pct_of_dense_bf16_peak"] = round(100.0 * tf / DENSE_BF16_SPEC_TFLOPS, 2)
+        res["roofline"] = {"bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
+                           "frac": round(tf / peak, 4), "peak_source": "measured bf16 burst (cuBLAS)"}
+    else:
+        res["kernel"] = "fwd_jvp_simt_f32_kernel<%d>" % w.D
+        res["bound"] = "launch latency (one launch of %d CTAs; fp32 CUDA-core path for the 1e-5 tolerance)" % (
+            w.B * w.H * ((w.N + 127) // 128))
+    in_bytes = 6 * w.B * w.H * w.N * w.D * ins[0].element_size()
+    res["l2"] = ("inputs larger than L2 (%.2f GB per step)" % (in_bytes / 1e9) if in_bytes > 126e6
+                 else "inputs L2-resident (%.1f KB; a parity-size case timed for completeness)" % (in_bytes / 1e3))
+    del ins, o, to, lse, tlse
+    torch.cuda.empty_cache()
+    if not with_cpu:
+        return res
+    ctf, dt, nrows, threads, desc = time_oracle(w, target_s=cpu_target_s, host_inputs=host)
+    res["cpu_baseline"] = {"value": round(ctf, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                           "sample": desc, "seconds": round(dt, 2), "rows_per_s": round(nrows / dt, 1),
+                           "extrapolated_full_call_s": round(fl / (ctf * 1e12), 2)}
+    return res
+
+
 # ------------------------------------------------------------------ GPU arm
-def bench_e2e(args, w, host, fl, world, stream, dev, barrier):
+def bench_e2e(args, w, host, fl_job, world, stream, dev, barrier):
     """Same metric through the public API from pinned host buffers: every step
-    copies the six inputs host->device and the four outputs device->host."""
+    copies this rank's six inputs host->device and its four outputs
+    device->host (attn_fwd_jvp on CPU tensors: the host-buffer entry point,
+    which overlaps the copies with the kernels chunk by chunk). Timed over
+    the same number of steps as the headline, clocks sampled meanwhile."""
     import masked_attention_jvp_b200 as caj
     pinned = [t.pin_memory() for t in host]
     h2d = sum(t.numel() * t.element_size() for t in pinned)
-    n_rows = w.B * w.H * w.N
-    d2h = 2 * n_rows * w.D * pinned[0].element_size() + 2 * n_rows * 4
-    steps = max(1, min(args.steps, 5))
-    caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)  # warm the host path once
+    n_rows = pinned[0].shape[0] * pinned[0].shape[1] * pinned[0].shape[2]
+    d2h = 2 * n_rows * pinned[0].shape[3] * pinned[0].element_size() + 2 * n_rows * 4
+    steps = args.steps
+    have_work = pinned[0].numel() > 0
+    if have_work:
+        caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)  # warm the host path once
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            if have_work:
+                caj.attn_fwd_jvp(*pinned, w.mask, scale=w.scale)
+        e1.record(stream)
+        torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    return {"value": round(whole_job_tflops(fl, world, steps, ms), 2), "unit": "TFLOP/s",
+    return {"value": round(strong_tflops(fl_job, steps, ms), 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3)}
+            "ms_per_step": round(ms / steps, 3), "clocks": clk.summary(),
+            "api": "attn_fwd_jvp on pinned CPU tensors (caj_attn_fwd_jvp_host)"}
+
+
+def rank_inputs(args, w, host, world, rank):
+    """This rank's share of the workload's inputs (host tensors) and the
+    problem it runs, by the split mode."""
+    if world == 1 or args.split == "replicas":
+        return host, w
+    if args.split == "heads":
+        h0, h1 = split_heads(w.H, world, rank)
+        return [t[:, h0:h1].contiguous() for t in host], w
+    # ulysses: this rank's sequence shard of every head
+    Ls = w.N // world
+    return [t[:, :, rank * Ls:(rank + 1) * Ls].contiguous() for t in host], w
 
 
 def bench_gpu(args, rank, world, local_rank):
@@ -510,21 +618,38 @@ def bench_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = selected_workload(args)
-    host = make_inputs(w, "cpu")
+    if args.split == "ulysses" and (w.H % world or w.N % world):
+        raise SystemExit(f"--split ulysses needs heads ({w.H}) and tokens ({w.N}) divisible by {world} ranks")
+    host_all = make_inputs(w, "cpu")
     if args.clean_tangent_zero:
         from masked_attention_jvp_b200.workloads import zero_clean_tangents
-        zero_clean_tangents(w, *host[3:])
+        zero_clean_tangents(w, *host_all[3:])
+    host, _ = rank_inputs(args, w, host_all, world, rank)
     ins = [t.to(dev) for t in host]
-    o = torch.empty_like(ins[0])
-    to = torch.empty_like(ins[0])
-    lse = torch.empty(ins[0].shape[:3], dtype=torch.float32, device=dev)
-    tlse = torch.empty_like(lse)
     stream = torch.cuda.current_stream(dev)
-    fl = flops_of(w)
+    fl = flops_of(w)                                   # one copy of the whole problem
+    fl_job = fl * (world if args.split == "replicas" else 1)
+    have_work = ins[0].numel() > 0
 
-    def step():
-        caj.attn_fwd_jvp_out(*ins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream,
-                             clean_tangent_zero=args.clean_tangent_zero)
+    if args.split == "ulysses" and world > 1:
+        from masked_attention_jvp_b200.ulysses import ulysses_attn_fwd_jvp
+
+        def step():
+            ulysses_attn_fwd_jvp(*ins, w.mask, scale=w.scale, clean_tangent_zero=args.clean_tangent_zero,
+                                 fused_output=args.fused_output)
+        launches_per_step = None  # NCCL kernels besides the library's
+    else:
+        o = torch.empty_like(ins[0])
+        to = torch.empty_like(ins[0])
+        lse = torch.empty(ins[0].shape[:3], dtype=torch.float32, device=dev)
+        tlse = torch.empty_like(lse)
+
+        def step():
+            if have_work:
+                caj.attn_fwd_jvp_out(*ins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream,
+                                     clean_tangent_zero=args.clean_tangent_zero)
+        L = w.mask.n_frames * w.mask.tokens_per_frame
+        launches_per_step = (2 if args.clean_tangent_zero and L >= 128 else 1) if have_work else 0
 
     for _ in range(args.warmup):
         step()
@@ -549,40 +674,64 @@ def bench_gpu(args, rank, world, local_rank):
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev)
     ms_per_step = total_ms / args.steps
-    value = whole_job_tflops(fl, world, args.steps, total_ms)
+    value = strong_tflops(fl_job, args.steps, total_ms)
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
-        e2e = bench_e2e(args, w, host, fl, world, stream, dev, barrier)
+    if not args.no_e2e and args.split != "ulysses":
+        e2e = bench_e2e(args, w, host, fl_job, world, stream, dev, barrier)
     if rank != 0:
         return None
     peaks, src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     kernel_ms = statistics.mean(per)
-    achieved = fl / (kernel_ms / 1e3) / 1e12
+    rank0_flops = fl if (world == 1 or args.split == "replicas") else fl * (
+        (split_heads(w.H, world, 0)[1] - split_heads(w.H, world, 0)[0]) / w.H if args.split == "heads" else 1.0 / world)
+    achieved = rank0_flops / (kernel_ms / 1e3) / 1e12
     clocks = clk.summary()
+    parallelism = {"heads": f"head split over {world} GPUs", "replicas": f"replica x{world}",
+                   "ulysses": f"Ulysses context parallelism over {world} GPUs"
+                              + (" (output all-to-all in the epilogue)" if args.fused_output else "")}[args.split]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak" if args.split == "replicas" else "strong",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) q,k,v; N(0,0.5^2) tangents)",
-        "config": workload_config(w, {"parallelism": f"replica x{world}" if world > 1 else "single GPU"}),
+        "config": workload_config(w, {"parallelism": parallelism if world > 1 else "single GPU"}),
         "pct_of_dense_bf16_peak": round(100.0 * value / world / DENSE_BF16_SPEC_TFLOPS, 2),
         "ms_per_step_min": round(min(per), 4), "ms_per_step_median": round(statistics.median(per), 4),
         "ms_per_step_each": [round(x, 3) for x in per],
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": launches_per_step * args.steps if launches_per_step is not None else None,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4),
                      "frac_of_sustained": round(achieved / peak_sustained, 4),
                      "peak_sustained": peak_sustained,
-                     "traffic": MEASURED_TRAFFIC.get((w.name, kernel_sources_hash())),
+                     "traffic": MEASURED_TRAFFIC.get((w.name, kernel_sources_hash())) if world == 1 else None,
                      "kernel_sources_sha256": kernel_sources_hash(),
                      "peak_source": f"{src} bf16 burst (cuBLAS)", "kernel": "fwd_jvp_sm100_kernel<128>"},
     }
+    if world > 1:
+        line["config"]["split"] = args.split
+        if args.split == "heads":
+            line["config"]["heads_per_rank"] = [b - a for a, b in (split_heads(w.H, world, r) for r in range(world))]
+        if args.split == "ulysses" and args.fused_output:
+            line["roofline"]["kernel"] = "fwd_jvp_sm100_kernel<128, scatter>"
+    if args.clean_tangent_zero:
+        line["roofline"]["traffic"] = None  # DRAM traffic was captured on dense inputs
+        line["roofline"]["kernel"] = "fwd_jvp_sm100_kernel<128, noisy and clean tile kinds>"
+        line["config"]["clean_tangent_zero"] = True
+        line["products_tflop_per_step"] = round(ctz_product_flops(w) / 1e12, 3)
+        line["roofline"]["achieved"] = round(ctz_product_flops(w) * rank0_flops / fl / (kernel_ms / 1e3) / 1e12, 2)
+        line["roofline"]["frac"] = round(line["roofline"]["achieved"] / peak, 4)
+        line["roofline"]["frac_of_sustained"] = round(line["roofline"]["achieved"] / peak_sustained, 4)
+        line["roofline"]["note"] = "achieved counts only the products the kernel must do"
+    if world > 1:
+        return line   # the single-GPU legs below run at N = 1 only
+
     if not args.no_backward and not args.clean_tangent_zero:
         line["backward"] = bench_backward(w, ins, o, lse, args.steps, peaks)
         line["gpu_launches_backward"] = 3 * args.steps
@@ -593,31 +742,30 @@ def bench_gpu(args, rank, world, local_rank):
         line["out_proj"] = bench_out_proj(w, dev, args.steps, peaks)
     if w.mask.tf_layout and not args.clean_tangent_zero and not args.no_ctz:
         line["clean_tangent_zero"] = bench_ctz(w, ins, args.steps, fl)
-    # last: it heats the GPU, and the legs above keep their earlier conditions
+    # last among the C2 legs: it heats the GPU, and the legs above keep their earlier conditions
     if not args.no_cp_scatter and not args.clean_tangent_zero:
         cp = bench_cp_scatter(w, ins, args.steps, fl)
         if cp is not None:
             line["cp_scatter"] = cp
             line["gpu_launches_cp_scatter"] = 2 * 4 * max(2, args.steps // 4)
-    if args.clean_tangent_zero:
-        # one launch for the query tiles with a noisy row, one for the clean ones
-        L = w.mask.n_frames * w.mask.tokens_per_frame
-        line["gpu_launches"] = args.steps * (2 if L >= 128 else 1)
-        line["roofline"]["traffic"] = None  # DRAM traffic was captured on dense inputs
-        line["roofline"]["kernel"] = "fwd_jvp_sm100_kernel<128, noisy and clean tile kinds>"
-        line["config"]["clean_tangent_zero"] = True
-        line["products_tflop_per_step"] = round(ctz_product_flops(w) / 1e12, 3)
-        line["roofline"]["achieved"] = round(ctz_product_flops(w) / (kernel_ms / 1e3) / 1e12, 2)
-        line["roofline"]["frac"] = round(line["roofline"]["achieved"] / peak, 4)
-        line["roofline"]["frac_of_sustained"] = round(line["roofline"]["achieved"] / peak_sustained, 4)
-        line["roofline"]["note"] = "achieved counts only the products the kernel must do"
-    if world == 1 and not args.no_cpu_baseline:
-        tf, dt, nrows, threads, desc = time_oracle(w, host_inputs=host)
+    if not args.no_cpu_baseline:
+        tf, dt, nrows, threads, desc = time_oracle(w, host_inputs=host_all)
         line["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": threads,
                                 "kind": "oracle", "sample": desc, "seconds": round(dt, 2),
                                 "rows_per_s": round(nrows / dt, 1),
                                 "extrapolated_full_call_s": round(fl / (tf * 1e12), 1),
                                 "host": host_cpu()}
+    if not args.no_configs and args.heads is None and not args.clean_tangent_zero:
+        del ins, o, to, lse, tlse
+        torch.cuda.empty_cache()
+        line["configs"] = {}
+        for name in WORKLOADS:
+            if name == w.name:
+                continue
+            line["configs"][name] = bench_config(name, args.steps, args.warmup, peaks,
+                                                 with_cpu=not args.no_cpu_baseline)
+            torch.cuda.empty_cache()
+        line["gpu_launches_configs"] = sum(c["gpu_launches"] for c in line["configs"].values())
     return line
 
 
@@ -678,6 +826,13 @@ def main():
                     help="skip the context-parallel output-scatter measurement")
     ap.add_argument("--no-ctz", action="store_true",
                     help="skip the clean-tangent-zero sub-measurement (teacher-forcing workloads)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other four workloads (the 'configs' key)")
+    ap.add_argument("--split", default="heads", choices=["heads", "replicas", "ulysses"],
+                    help="multi-GPU work split: the problem's heads over the ranks (default, strong scaling), "
+                         "a copy per rank (weak scaling), or Ulysses sequence shards with all-to-alls")
+    ap.add_argument("--fused-output", action="store_true",
+                    help="with --split ulysses: the output all-to-all in the attention epilogue")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (small cases for ncu section captures)")
     ap.add_argument("--clean-tangent-zero", action="store_true",

@@ -146,8 +146,10 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v,
  * orders every rank's reads after all P calls, e.g. with a barrier on the
  * stream. The buffers are owned by the caller.
  * Returns as caj_attn_fwd_jvp. CAJ_ERR_INVALID_ARG is also returned for a null
- * dst, a shard count or head range out of bounds, or a null or misaligned
- * slice pointer.
+ * dst, a shard count or head range out of bounds, a null or misaligned slice
+ * pointer, or a slice pointer that is not device memory (host memory, pinned
+ * or not, by cudaPointerGetAttributes): the kernel writes the slices with
+ * device stores.
  */
 #define CAJ_MAX_SHARDS 8
 typedef struct {
@@ -163,6 +165,35 @@ caj_status caj_attn_fwd_jvp_scatter(const void *q, const void *k, const void *v,
                                     const void *tq, const void *tk, const void *tv,
                                     const caj_problem *prob, const caj_mask_desc *mask,
                                     const caj_seq_scatter *dst, void *stream);
+
+/*
+ * Stream-ordered barrier of the P ranks of a context-parallel group, the fence
+ * around caj_attn_fwd_jvp_scatter (section 3.2.2, "JVP Ulysses CP": the output
+ * all-to-all; here every rank writes rows into its peers' memory, so each rank
+ * must know when its peers have finished reading, and later writing, its slice).
+ *   pads[r]     device pointer, as mapped in this process, to rank r's pad of
+ *               CAJ_MAX_SHARDS uint32 words (symmetric memory or CUDA IPC with
+ *               peer access; pads[rank] is this rank's own). Every pad starts
+ *               zeroed before any rank's first call.
+ *   shards      P, 1..CAJ_MAX_SHARDS;  rank: this rank, 0..P-1
+ *   epoch       nonzero, larger than on any earlier call over these pads
+ *               (wrapping compare: a counter from 1 serves for 2^31 calls);
+ *               every rank passes the same value to the same barrier
+ *   timeout_ms  limit on the wait; <= 0 takes the library's wait limit
+ *               (caj_set_wait_timeout_ms)
+ * One small kernel on `stream`: rank r stores `epoch` into word r of every
+ * rank's pad (system-scope release, after a system fence that orders this
+ * rank's earlier work on the stream before it), then waits until every word of
+ * its own pad has reached `epoch` (system-scope acquire). Work enqueued on
+ * `stream` after the call starts once every rank has arrived. The wait is
+ * bounded: if a peer does not arrive in time the kernel records
+ * CAJ_ERR_DEVICE_TIMEOUT (caj_last_device_error_code 0x1F0), read by
+ * caj_last_device_status, and returns; it never traps.
+ * Returns CAJ_OK once enqueued, CAJ_ERR_INVALID_ARG (null or misaligned pad,
+ * rank or shard count out of range, epoch 0) without launching, or CAJ_ERR_CUDA.
+ */
+caj_status caj_signal_barrier(uint32_t *const *pads, int32_t shards, int32_t rank, uint32_t epoch,
+                              double timeout_ms, void *stream);
 
 /*
  * Host-buffer form of caj_attn_fwd_jvp: the same operation, with the inputs
@@ -309,7 +340,8 @@ caj_status caj_last_device_status(void *stream);
 
 /* Detail of the last device error (0 if none). Valid after
  * caj_last_device_status returned CAJ_ERR_DEVICE_TIMEOUT:
- *   0x100 | site   a bounded wait expired at the numbered wait site;
+ *   0x100 | site   a bounded wait expired at the numbered wait site (site 0xF0:
+ *                  the signal barrier, caj_signal_barrier);
  *   0x200          the dynamic shared memory was not 1 KiB aligned;
  *   0x300          a forward launch met a query tile of the other kind than it
  *                  was built for (an internal partitioning error). */

@@ -28,7 +28,7 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "signal_barrier", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -233,6 +233,10 @@ def attn_fwd_jvp_scatter(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, head_base:
     Ls = N // P
     out_shape = (B, Ls, Ht, D) if token_major_out else (B, Ht, Ls, D)
     for r in range(P):
+        for t in (o[r], to[r], lse[r], tlse[r]):
+            if not t.is_cuda:
+                raise ValueError(f"attn_fwd_jvp_scatter: slice {r} buffers must be CUDA tensors "
+                                 "(the kernel writes them with device stores)")
         for t in (o[r], to[r]):
             if t.dtype != q.dtype or tuple(t.shape) != out_shape or not t.is_contiguous():
                 raise ValueError(f"attn_fwd_jvp_scatter: slice {r} output must be contiguous {out_shape}")
@@ -250,6 +254,23 @@ def attn_fwd_jvp_scatter(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, head_base:
                                              ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)),
                                              ctypes.byref(dst), ctypes.c_void_p(s))
     _lib.check(st, "caj_attn_fwd_jvp_scatter")
+
+
+def signal_barrier(pads, rank: int, epoch: int, timeout_ms: float = 0.0,
+                   stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Stream-ordered barrier of the P ranks of a context-parallel group
+    (caj_signal_barrier). pads: P device addresses (ints), entry r rank r's pad
+    of MAX_SHARDS uint32 words as mapped in this process, zeroed before the
+    first call. epoch: the same nonzero value on every rank, larger than any
+    earlier one over these pads. A peer that does not arrive within timeout_ms
+    (<= 0: the library's wait limit) makes the kernel record a timeout, which
+    device_status() raises; the kernel never traps."""
+    P = len(pads)
+    arr = (ctypes.c_void_p * max(P, 1))(*[int(p) for p in pads])
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    st = _lib.lib().caj_signal_barrier(arr, P, int(rank), ctypes.c_uint32(int(epoch) & 0xFFFFFFFF),
+                                       float(timeout_ms), ctypes.c_void_p(s))
+    _lib.check(st, "caj_signal_barrier")
 
 
 def out_proj_jvp(x, tx, w, bias=None, out=None):

@@ -18,7 +18,7 @@ EXPORTED = [
     "caj_row_key_ranges", "caj_qtile_key_tiles", "caj_version", "caj_set_wait_timeout_ms",
     "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
     "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host", "caj_out_proj_jvp",
-    "caj_attn_fwd_jvp_scatter", "caj_attn_fwd_jvp_host_static",
+    "caj_attn_fwd_jvp_scatter", "caj_attn_fwd_jvp_host_static", "caj_signal_barrier",
 ]
 
 
@@ -120,6 +120,8 @@ def lib() -> ctypes.CDLL:
         L.caj_attn_fwd_jvp_scatter.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC),
                                                 ctypes.POINTER(SeqScatterC), vp]
         L.caj_attn_fwd_jvp_scatter.restype = ctypes.c_int
+        L.caj_signal_barrier.argtypes = [ctypes.POINTER(vp), i32, i32, ctypes.c_uint32, ctypes.c_double, vp]
+        L.caj_signal_barrier.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcausaljvp.so")
 SOURCES = ["api.cpp", "fwd_jvp_sm100.cu", "fwd_jvp_simt.cu", "prologue.cu", "bwd_sm100.cu",
-           "host_static.cu"]
+           "host_static.cu", "signal.cu"]
 HEADERS = ["kernels.h", "mask_schedule.h", "ptx_sm100.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -486,6 +486,20 @@ caj_status caj_attn_fwd_jvp_scatter(const void *q, const void *k, const void *v,
   }
   st = check_device();
   if (st != CAJ_OK) return st;
+  // the epilogue writes the slices with device stores: host memory (pinned or
+  // not) is refused here rather than met by the kernel
+  for (int32_t r = 0; r < dst->shards; ++r) {
+    const void *slice[4] = {dst->o[r], dst->to[r], dst->lse[r], dst->tlse[r]};
+    for (const void *ptr : slice) {
+      cudaPointerAttributes a{};
+      cudaError_t e = cudaPointerGetAttributes(&a, ptr);
+      if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // the failed query leaves its error behind: clear it
+        return CAJ_ERR_INVALID_ARG;
+      }
+      if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return CAJ_ERR_INVALID_ARG;
+    }
+  }
 
   caj::OutMap out{};
   for (int32_t r = 0; r < dst->shards; ++r) {
@@ -694,13 +708,35 @@ caj_status caj_attn_bwd(const void *q, const void *k, const void *v, const void 
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
 }
 
+caj_status caj_signal_barrier(uint32_t *const *pads, int32_t shards, int32_t rank, uint32_t epoch,
+                              double timeout_ms, void *stream) {
+  if (!pads || shards < 1 || shards > CAJ_MAX_SHARDS || rank < 0 || rank >= shards || epoch == 0)
+    return CAJ_ERR_INVALID_ARG;
+  caj::SignalParams p{};
+  for (int32_t r = 0; r < shards; ++r) {
+    if (!pads[r] || !aligned4(pads[r])) return CAJ_ERR_INVALID_ARG;
+    p.pads[r] = pads[r];
+  }
+  caj_status st = check_device();
+  if (st != CAJ_OK) return st;
+  p.shards = shards;
+  p.rank = rank;
+  p.epoch = epoch;
+  p.timeout_ns = timeout_ms > 0.0 ? uint64_t(timeout_ms * 1e6) : wait_timeout_ns();
+  cudaError_t e = caj::launch_signal_barrier(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+}
+
 caj_status caj_last_device_status(void *stream) {
-  uint32_t code = 0, bcode = 0;
+  uint32_t code = 0, bcode = 0, scode = 0;
   cudaError_t e = caj::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &code);
   if (e != cudaSuccess) return cuda_fail(e);
   e = caj::read_and_clear_bwd_error(&bcode);
   if (e != cudaSuccess) return cuda_fail(e);
+  e = caj::read_and_clear_signal_error(&scode);
+  if (e != cudaSuccess) return cuda_fail(e);
   if (!code) code = bcode;
+  if (!code) code = scode;
   if (code != 0) {
     g_last_device_code = code;
     return CAJ_ERR_DEVICE_TIMEOUT;

@@ -24,6 +24,9 @@ enum DeviceError : uint32_t {
   kErrTileKind = 0x300,        // a query tile outside the kind its launch covers
 };
 
+// Wait site of the signal barrier (kErrTimeoutBase | site when it gives up).
+constexpr uint32_t kSiteSignalBarrier = 0xF0;
+
 // Query tiles of one launch of the tensor-core forward. With clean-tangent-zero
 // teacher forcing (tq, tk, tv vanish on rows < L) a call runs as two launches,
 // one per kind of query tile: each kernel instantiation carries only its own
@@ -140,12 +143,23 @@ struct BwdParams {
   int32_t fault_mode;     // test hook: 1 = the producers issue no copies
 };
 
+// Signal barrier of a context-parallel group: pads[r] is rank r's pad of
+// kMaxShards words as mapped in this process.
+struct SignalParams {
+  uint32_t *pads[kMaxShards];
+  int32_t shards, rank;
+  uint32_t epoch;
+  uint64_t timeout_ns;
+};
+
 // Each returns the launch's cudaError_t (cudaSuccess when enqueued).
 cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream);
 cudaError_t launch_fwd_jvp_simt_f32(const SimtParams &p, int D, cudaStream_t stream);
 cudaError_t launch_qk_norm_rope_jvp(const PrologueParams &p, cudaStream_t stream);
 cudaError_t launch_attn_bwd_sm100(const BwdParams &p, int D, cudaStream_t stream);
 cudaError_t read_and_clear_bwd_error(uint32_t *out);
+cudaError_t launch_signal_barrier(const SignalParams &p, cudaStream_t stream);
+cudaError_t read_and_clear_signal_error(uint32_t *out);
 
 // Device error word access (defined next to the kernels that write it).
 cudaError_t read_and_clear_device_error(cudaStream_t stream, uint32_t *out);

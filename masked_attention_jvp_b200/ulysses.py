@@ -68,9 +68,10 @@ def head_to_seq(y: torch.Tensor, group=None) -> torch.Tensor:
 class SliceBuffers:
     """This rank's output slice in symmetric memory, mapped on every rank.
 
-    One allocation holds O, tO [B, H, Ls, D] and LSE, tLSE [B, H, Ls] fp32
-    (regions 256-byte aligned). o[r], to[r], lse[r], tlse[r] view rank r's copy:
-    rank r's device memory, reached over NVLink for r != this rank."""
+    One allocation holds O, tO [B, H, Ls, D], LSE, tLSE [B, H, Ls] fp32 and a
+    pad of signal words for the barrier (regions 256-byte aligned). o[r],
+    to[r], lse[r], tlse[r] view rank r's copy: rank r's device memory, reached
+    over NVLink for r != this rank."""
 
     def __init__(self, B: int, H: int, Ls: int, D: int, dtype: torch.dtype, device, group=None):
         import torch.distributed._symmetric_memory as symm_mem
@@ -81,9 +82,14 @@ class SliceBuffers:
         es = torch.empty((), dtype=dtype).element_size()
         n_out, n_st = B * H * Ls * D, B * H * Ls
         offs = [0, up(n_out * es), 2 * up(n_out * es), 2 * up(n_out * es) + up(n_st * 4)]
-        total = offs[3] + up(n_st * 4)
+        pad_off = offs[3] + up(n_st * 4)
+        total = pad_off + 256
         self.key = (B, H, Ls, D, dtype, torch.device(device))
         self.buf = symm_mem.empty(total, dtype=torch.uint8, device=device)
+        # the signal pad starts at zero before any peer can reach it: the
+        # rendezvous below is the first point where peers learn its address
+        self.buf.zero_()
+        torch.cuda.synchronize(device)
         self.handle = symm_mem.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
         self.rank, self.world = self.handle.rank, self.handle.world_size
         hd = self.handle
@@ -96,10 +102,18 @@ class SliceBuffers:
         self.to = [view(r, offs[1], (B, H, Ls, D), dtype) for r in range(P)]
         self.lse = [view(r, offs[2], (B, H, Ls), torch.float32) for r in range(P)]
         self.tlse = [view(r, offs[3], (B, H, Ls), torch.float32) for r in range(P)]
+        self.pads = [view(r, pad_off, (64,), torch.int32).data_ptr() for r in range(P)]
+        self.epoch = 0
 
     def barrier(self, timeout_ms: int = 10000):
-        """Stream-ordered barrier over the group's ranks."""
-        self.handle.barrier(channel=0, timeout_ms=timeout_ms)
+        """Stream-ordered barrier over the group's ranks: the library's signal
+        kernel over the mapped pads (caj_signal_barrier). A peer that does not
+        arrive within timeout_ms makes the kernel record a timeout, which
+        masked_attention_jvp_b200.device_status() raises; nothing traps.
+        Every rank calls it the same number of times, so the epochs agree."""
+        from . import signal_barrier
+        self.epoch += 1
+        signal_barrier(self.pads, self.rank, self.epoch, timeout_ms)
 
 
 class _LocalSlices:
@@ -121,7 +135,9 @@ _slice_buffers = {}
 
 
 def _get_slice_buffers(B, H, Ls, D, dtype, device, group):
-    key = (B, H, Ls, D, dtype, torch.device(device), id(group))
+    # whether a process group exists, and its size, are part of the key: local
+    # slices made before init_process_group never serve a group afterwards
+    key = (B, H, Ls, D, dtype, torch.device(device), id(group), dist.is_initialized(), _world(group))
     sb = _slice_buffers.get(key)
     if sb is None:
         if dist.is_initialized():
@@ -149,7 +165,9 @@ def ulysses_attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = Non
     symmetric-memory slice buffer of its owner (see SliceBuffers). The
     returned tensors are copies, so the slice buffers are free for the next
     call once every rank has passed its first barrier. Without a process group
-    (a single process) the one slice is ordinary device memory.
+    (a single process) the one slice is ordinary device memory. The barriers
+    are bounded: a peer that never arrives leaves a timeout status, raised by
+    masked_attention_jvp_b200.device_status(), not a trapped GPU.
     """
     ins = torch.stack([q, k, v, tq, tk, tv])
     if fused_output:

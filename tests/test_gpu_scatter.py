@@ -6,12 +6,22 @@ whole sequence and storing every row into the slice buffer of the token's
 owner. The P slice buffers are local here; on a multi-GPU run they are the
 ranks' memory and the same stores cross NVLink. The launches only store, they
 never wait on one another. After all P launches slice r must equal rows
-[r N/P, (r+1) N/P) of the direct call, bit for bit, for every head."""
+[r N/P, (r+1) N/P) of the direct call, bit for bit, for every head. The slices,
+put back together, must also match the fp64 oracle within the parity tests'
+tolerances (every row for the small cases; 512 seeded rows per head plus the
+chunk boundaries at full size), so a layout error shared by the direct and the
+scattering kernels cannot pass."""
+import ctypes
+
 import pytest
 import torch
 
+import oracle
+
 import masked_attention_jvp_b200 as caj
-from masked_attention_jvp_b200.workloads import MaskDesc, make_inputs, small, zero_clean_tangents
+from masked_attention_jvp_b200.workloads import (MaskDesc, boundary_rows, make_inputs, sample_rows, small,
+                                                 zero_clean_tangents)
+from tests.test_gpu_parity import check_rows, gather
 
 pytestmark = pytest.mark.gpu
 
@@ -39,6 +49,16 @@ def _rows(t, rows, token_major):
     return t[:, rows] if token_major else t[:, :, rows]
 
 
+def _assemble(o, to, lse, tlse, token_major):
+    """The P slices put back together as [B, H, N, D] and [B, H, N]."""
+    if token_major:
+        fo = torch.cat(o, dim=1).permute(0, 2, 1, 3).contiguous()
+        fto = torch.cat(to, dim=1).permute(0, 2, 1, 3).contiguous()
+    else:
+        fo, fto = torch.cat(o, dim=2), torch.cat(to, dim=2)
+    return fo, fto, torch.cat(lse, dim=2), torch.cat(tlse, dim=2)
+
+
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_scatter_equals_direct_call(case):
     name, B, H, D, mask, dtype, P, ctz, tm = case
@@ -61,6 +81,10 @@ def test_scatter_equals_direct_call(case):
         assert torch.equal(to[r], _rows(direct[1], rows, tm)), (name, r, "to")
         assert torch.equal(lse[r], direct[2][:, :, rows]), (name, r, "lse")
         assert torch.equal(tlse[r], direct[3][:, :, rows]), (name, r, "tlse")
+    # every row of the reassembled slices against the oracle
+    ref = oracle.attn_fwd_jvp_rows(*[t.cpu() for t in ins], w.mask)
+    full = _assemble(o, to, lse, tlse, tm)
+    check_rows(gather(full, torch.arange(B * H * N), D), ref, dtype, name)
 
 
 def test_scatter_writes_only_its_own_heads():
@@ -114,3 +138,40 @@ def test_scatter_at_full_size_equals_direct_call():
         assert torch.equal(to[r], direct[1][:, :, rows])
         assert torch.equal(lse[r], direct[2][:, :, rows])
         assert torch.equal(tlse[r], direct[3][:, :, rows])
+    del direct
+    full = _assemble(o, to, lse, tlse, False)
+    del o, to, lse, tlse
+    rows = torch.unique(torch.cat([sample_rows(w, 512, seed_offset=9), boundary_rows(w)]))
+    got = gather(full, rows, w.D)
+    host = [t.cpu() for t in ins]
+    del ins, full
+    ref = oracle.attn_fwd_jvp_rows(*host, w.mask, rows=rows)
+    check_rows(got, ref, w.dtype, "scatter full size")
+
+
+def test_scatter_refuses_host_memory_slices():
+    """Slices in host memory are refused before any launch: by the Python
+    binding (CPU tensors), and by the library itself for pinned host memory
+    given through the C-ABI (device-reachable, so nothing could fault even if
+    the check were missing; the status is what is checked)."""
+    w = small("host_slices", 1, 2, 64, MaskDesc(16, 1, 4, 0), bf, seed=34)
+    ins = make_inputs(w, "cuda")
+    o, to, lse, tlse = _slices(1, 2, 32, 64, bf, 2, False)
+    cpu_o = [t.cpu() for t in o]
+    with pytest.raises(ValueError):
+        caj.attn_fwd_jvp_scatter(*ins, w.mask, cpu_o, to, lse, tlse)
+    pinned = torch.zeros(1, 2, 32, 64, dtype=bf).pin_memory()
+    dst = caj._lib.SeqScatterC()
+    dst.shards, dst.head_base, dst.heads_total = 2, 0, 2
+    for r in range(2):
+        dst.o[r], dst.to[r] = o[r].data_ptr(), to[r].data_ptr()
+        dst.lse[r], dst.tlse[r] = lse[r].data_ptr(), tlse[r].data_ptr()
+    dst.to[1] = pinned.data_ptr()
+    prob = caj._problem(ins[0], None)
+    st = caj._lib.lib().caj_attn_fwd_jvp_scatter(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
+                                                 ctypes.byref(prob), ctypes.byref(caj._lib.mask_c(w.mask)),
+                                                 ctypes.byref(dst), None)
+    torch.cuda.synchronize()
+    assert st == caj._lib.CAJ_ERR_INVALID_ARG
+    assert torch.count_nonzero(pinned.float()) == 0
+    assert all(torch.isnan(t.float()).all() for t in o)  # nothing launched

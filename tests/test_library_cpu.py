@@ -22,6 +22,12 @@ MASKS = [MaskDesc(3, 1, 4, 0), MaskDesc(2, 2, 4, 0), MaskDesc(3, 1, 3, 1), MaskD
          MaskDesc(13, 3, 6, 1), MaskDesc(64, 1, 4, 1), MaskDesc(1, 1, 130, 1)]
 
 
+
+# Calls whose arguments pass validation reach the device check: on a machine
+# without a GPU they stop there (CAJ_ERR_CUDA); elsewhere they would launch
+# with the fake pointers these tests use, so they run only without a GPU.
+_NO_GPU = not torch.cuda.is_available()
+
 def test_header_symbols_are_exported():
     hdr = open(os.path.join(ROOT, "include", "causaljvp.h")).read()
     declared = sorted(set(re.findall(r"\b(caj_[a-z_]+)\s*\(", hdr)))
@@ -124,12 +130,14 @@ def test_argument_validation_launches_nothing():
     assert _call(mask=M(16, 3, 4, 0)) == INV                   # frames % chunk != 0
     assert _call(mask=M(16, 1, 4, 2)) == INV                   # bad layout flag
     assert _call(mask=M(0, 1, 4, 0)) == INV                    # empty frame
-    assert _call(prob=P(1, 2, 128, 64, bf, 0.0), mask=M(16, 1, 4, 1)) != INV  # TF: N = 2L
+    if _NO_GPU:  # would launch with these fake pointers on a GPU machine
+        assert _call(prob=P(1, 2, 128, 64, bf, 0.0), mask=M(16, 1, 4, 1)) != INV  # TF: N = 2L
     assert _call(prob=P(1, 2, 64, 96, bf, 0.0)) == UNS         # head dim not built
     assert _call(prob=P(700, 100, 64, 64, bf, 0.0)) == UNS     # too many heads
     assert _call(prob=P(1, 2, 64, 64, bf, 0.0, 1)) == INV      # clean-tangent flag needs TF layout
     assert _call(prob=P(1, 2, 64, 64, bf, 0.0, 4)) == INV      # unknown flag bit
-    assert _call(prob=P(1, 2, 128, 64, bf, 0.0, 1), mask=M(16, 1, 4, 1)) != INV
+    if _NO_GPU:  # would launch with these fake pointers on a GPU machine
+        assert _call(prob=P(1, 2, 128, 64, bf, 0.0, 1), mask=M(16, 1, 4, 1)) != INV
 
 
 def _ws_bytes(prob):
@@ -279,8 +287,10 @@ def test_out_proj_validation_launches_nothing():
 def test_token_major_flag_validation():
     P, M = _lib.ProblemC, _lib.MaskDescC
     bf, tm, ctz = _lib.CAJ_DTYPE_BF16, _lib.CAJ_FLAG_TOKEN_MAJOR_OUT, _lib.CAJ_FLAG_CLEAN_TANGENT_ZERO
-    assert _call(prob=P(1, 2, 64, 64, bf, 0.0, tm)) != _lib.CAJ_ERR_INVALID_ARG      # accepted
-    assert _call(prob=P(1, 2, 128, 64, bf, 0.0, tm | ctz), mask=M(16, 1, 4, 1)) != _lib.CAJ_ERR_INVALID_ARG
+    if _NO_GPU:  # would launch with these fake pointers on a GPU machine
+        assert _call(prob=P(1, 2, 64, 64, bf, 0.0, tm)) != _lib.CAJ_ERR_INVALID_ARG      # accepted
+    if _NO_GPU:  # would launch with these fake pointers on a GPU machine
+        assert _call(prob=P(1, 2, 128, 64, bf, 0.0, tm | ctz), mask=M(16, 1, 4, 1)) != _lib.CAJ_ERR_INVALID_ARG
     assert _call(prob=P(1, 2, 64, 64, bf, 0.0, 8)) == _lib.CAJ_ERR_INVALID_ARG       # unknown bit
     # the host-buffer form copies head-major chunks only
     _, need = _ws_bytes(P(1, 2, 64, 64, bf, 0.0))
@@ -319,9 +329,32 @@ def test_scatter_validation_launches_nothing():
     assert _scatter_call(o=0x20008) == INV                                   # misaligned O slice
     assert _scatter_call(lse=0x30002) == INV                                 # misaligned LSE slice
     assert _scatter_call(null_slice=1) == INV                                # a used slice is null
-    assert _scatter_call(shards=1, null_slice=1) != INV                      # an unused one may be
+    if _NO_GPU:  # would launch with these fake pointers on a GPU machine
+        assert _scatter_call(shards=1, null_slice=1) != INV                      # an unused one may be
     assert _scatter_call(prob=P(1, 2, 64, 64, bf, 0.0, 1)) == INV            # clean-tangent needs TF
     assert _scatter_call(prob=P(1, 2, 64, 96, bf, 0.0)) == _lib.CAJ_ERR_UNSUPPORTED
     for ok in (dict(shards=8, head_base=2), dict(shards=4, heads_total=2),
                dict(prob=P(1, 2, 64, 64, bf, 0.0, _lib.CAJ_FLAG_TOKEN_MAJOR_OUT))):
-        assert _scatter_call(**ok) != INV, ok
+        if _NO_GPU:  # would launch with these fake pointers on a GPU machine
+            assert _scatter_call(**ok) != INV, ok
+
+
+def test_signal_barrier_validation_launches_nothing():
+    L = _lib.lib()
+    INV = _lib.CAJ_ERR_INVALID_ARG
+    vp = ctypes.c_void_p
+
+    def call(pads, shards, rank, epoch):
+        arr = (vp * max(len(pads), 1))(*pads)
+        return L.caj_signal_barrier(arr, shards, rank, epoch, 0.0, vp(0))
+
+    assert L.caj_signal_barrier(None, 1, 0, 1, 0.0, vp(0)) == INV         # no pad list
+    assert call([0x1000], 0, 0, 1) == INV                                  # no rank
+    assert call([0x1000] * 9, 9, 0, 1) == INV                              # more ranks than a pad holds
+    assert call([0x1000, 0x2000], 2, 2, 1) == INV                          # rank out of range
+    assert call([0x1000, 0x2000], 2, -1, 1) == INV
+    assert call([0x1000, 0x2000], 2, 0, 0) == INV                          # epoch 0 is the pads' start value
+    assert call([0x1000, 0], 2, 0, 1) == INV                               # null pad
+    assert call([0x1000, 0x2002], 2, 0, 1) == INV                          # misaligned pad
+    if _NO_GPU:
+        assert call([0x1000, 0x2000], 2, 1, 7) == _lib.CAJ_ERR_CUDA        # valid: stops at the device check
