@@ -196,6 +196,32 @@ caj_status caj_signal_barrier(uint32_t *const *pads, int32_t shards, int32_t ran
                               double timeout_ms, void *stream);
 
 /*
+ * Peer mappings for the slice buffers of caj_attn_fwd_jvp_scatter (section
+ * 3.2.1 "Parallelism": each rank's output slice must be writable by every
+ * rank). Plain CUDA IPC: a rank exports a handle for device memory it owns,
+ * the other ranks open it as a peer mapping over NVLink. No multicast object
+ * is created or bound.
+ *   caj_ipc_export  ptr: device memory from cudaMalloc on the current device
+ *                   (e.g. PyTorch's default allocator; not memory from
+ *                   cudaMallocAsync or cuMemCreate). Writes an opaque handle
+ *                   (the allocation's IPC handle and ptr's offset inside it).
+ *   caj_ipc_open    maps a handle exported by ANOTHER process (same node) and
+ *                   returns the address of the exported ptr in this process;
+ *                   peer access is enabled on first touch.
+ *   caj_ipc_close   unmaps an address returned by caj_ipc_open. The exporter
+ *                   keeps its memory until every opener has closed it.
+ * Return CAJ_OK, CAJ_ERR_INVALID_ARG (null argument; an address not opened
+ * here) or CAJ_ERR_CUDA (caj_last_cuda_error names the CUDA error).
+ */
+typedef struct {
+  unsigned char handle[64];
+  uint64_t offset;
+} caj_ipc_handle;
+caj_status caj_ipc_export(const void *ptr, caj_ipc_handle *out);
+caj_status caj_ipc_open(const caj_ipc_handle *h, void **ptr);
+caj_status caj_ipc_close(void *ptr);
+
+/*
  * Host-buffer form of caj_attn_fwd_jvp: the same operation, with the inputs
  * and outputs in host memory. The heads are split into at most 16 chunks.
  * Three things run at once on three streams: the copy of chunk c's six inputs

@@ -28,7 +28,8 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "signal_barrier", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
+__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "signal_barrier",
+           "ipc_export", "ipc_open", "ipc_close", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -271,6 +272,34 @@ def signal_barrier(pads, rank: int, epoch: int, timeout_ms: float = 0.0,
     st = _lib.lib().caj_signal_barrier(arr, P, int(rank), ctypes.c_uint32(int(epoch) & 0xFFFFFFFF),
                                        float(timeout_ms), ctypes.c_void_p(s))
     _lib.check(st, "caj_signal_barrier")
+
+
+def ipc_export(t: torch.Tensor) -> bytes:
+    """An IPC handle (bytes) through which another process on this node maps
+    the device memory of CUDA tensor `t` (caj_ipc_export). `t` must come from
+    PyTorch's default cudaMalloc-backed allocator."""
+    if not t.is_cuda:
+        raise ValueError("ipc_export: a CUDA tensor is needed")
+    h = _lib.IpcHandleC()
+    _lib.check(_lib.lib().caj_ipc_export(ctypes.c_void_p(t.data_ptr()), ctypes.byref(h)), "caj_ipc_export")
+    return bytes(ctypes.string_at(ctypes.addressof(h), ctypes.sizeof(h)))
+
+
+def ipc_open(handle: bytes) -> int:
+    """Maps a handle from ipc_export of ANOTHER process; returns the device
+    address of the exported tensor's first byte in this process."""
+    h = _lib.IpcHandleC()
+    if len(handle) != ctypes.sizeof(h):
+        raise ValueError("ipc_open: not a handle from ipc_export")
+    ctypes.memmove(ctypes.addressof(h), handle, len(handle))
+    p = ctypes.c_void_p(0)
+    _lib.check(_lib.lib().caj_ipc_open(ctypes.byref(h), ctypes.byref(p)), "caj_ipc_open")
+    return int(p.value)
+
+
+def ipc_close(address: int) -> None:
+    """Unmaps an address returned by ipc_open."""
+    _lib.check(_lib.lib().caj_ipc_close(ctypes.c_void_p(int(address))), "caj_ipc_close")
 
 
 def out_proj_jvp(x, tx, w, bias=None, out=None):

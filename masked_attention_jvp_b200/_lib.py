@@ -19,6 +19,7 @@ EXPORTED = [
     "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
     "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host", "caj_out_proj_jvp",
     "caj_attn_fwd_jvp_scatter", "caj_attn_fwd_jvp_host_static", "caj_signal_barrier",
+    "caj_ipc_export", "caj_ipc_open", "caj_ipc_close",
 ]
 
 
@@ -30,6 +31,10 @@ class SeqScatterC(ctypes.Structure):
     _fields_ = [("shards", ctypes.c_int32), ("head_base", ctypes.c_int32), ("heads_total", ctypes.c_int32),
                 ("o", ctypes.c_void_p * MAX_SHARDS), ("to", ctypes.c_void_p * MAX_SHARDS),
                 ("lse", ctypes.c_void_p * MAX_SHARDS), ("tlse", ctypes.c_void_p * MAX_SHARDS)]
+
+
+class IpcHandleC(ctypes.Structure):
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64)]
 
 
 class LinearShapeC(ctypes.Structure):
@@ -122,6 +127,12 @@ def lib() -> ctypes.CDLL:
         L.caj_attn_fwd_jvp_scatter.restype = ctypes.c_int
         L.caj_signal_barrier.argtypes = [ctypes.POINTER(vp), i32, i32, ctypes.c_uint32, ctypes.c_double, vp]
         L.caj_signal_barrier.restype = ctypes.c_int
+        L.caj_ipc_export.argtypes = [vp, ctypes.POINTER(IpcHandleC)]
+        L.caj_ipc_export.restype = ctypes.c_int
+        L.caj_ipc_open.argtypes = [ctypes.POINTER(IpcHandleC), ctypes.POINTER(vp)]
+        L.caj_ipc_open.restype = ctypes.c_int
+        L.caj_ipc_close.argtypes = [vp]
+        L.caj_ipc_close.restype = ctypes.c_int
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

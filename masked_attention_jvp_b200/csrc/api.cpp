@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <memory>
 #include <mutex>
 #include <vector>
@@ -724,6 +725,70 @@ caj_status caj_signal_barrier(uint32_t *const *pads, int32_t shards, int32_t ran
   p.epoch = epoch;
   p.timeout_ns = timeout_ms > 0.0 ? uint64_t(timeout_ms * 1e6) : wait_timeout_ns();
   cudaError_t e = caj::launch_signal_barrier(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
+}
+
+namespace {
+using AddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+AddressRangeFn get_address_range() {
+  static std::once_flag once;
+  static AddressRangeFn fn = nullptr;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddressRangeFn>(ptr);
+  });
+  return fn;
+}
+
+// Addresses handed out by caj_ipc_open, with the mapped allocation's base.
+std::mutex g_ipc_mu;
+std::map<uintptr_t, void *> g_ipc_open;
+}  // namespace
+
+caj_status caj_ipc_export(const void *ptr, caj_ipc_handle *out) {
+  if (!ptr || !out) return CAJ_ERR_INVALID_ARG;
+  AddressRangeFn range = get_address_range();
+  if (!range) return cuda_fail(cudaErrorNotSupported);
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return CAJ_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base));
+  if (e != cudaSuccess) return cuda_fail(e);
+  static_assert(sizeof(h) == sizeof(out->handle), "IPC handle size");
+  std::memcpy(out->handle, &h, sizeof(h));
+  out->offset = uint64_t(reinterpret_cast<uintptr_t>(ptr) - uintptr_t(base));
+  return CAJ_OK;
+}
+
+caj_status caj_ipc_open(const caj_ipc_handle *h, void **ptr) {
+  if (!h || !ptr) return CAJ_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t ch;
+  std::memcpy(&ch, h->handle, sizeof(ch));
+  void *base = nullptr;
+  cudaError_t e = cudaIpcOpenMemHandle(&base, ch, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_fail(e);
+  void *p = static_cast<uint8_t *>(base) + h->offset;
+  std::lock_guard<std::mutex> lock(g_ipc_mu);
+  g_ipc_open[reinterpret_cast<uintptr_t>(p)] = base;
+  *ptr = p;
+  return CAJ_OK;
+}
+
+caj_status caj_ipc_close(void *ptr) {
+  void *base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_ipc_mu);
+    auto it = g_ipc_open.find(reinterpret_cast<uintptr_t>(ptr));
+    if (!ptr || it == g_ipc_open.end()) return CAJ_ERR_INVALID_ARG;
+    base = it->second;
+    g_ipc_open.erase(it);
+  }
+  cudaError_t e = cudaIpcCloseMemHandle(base);
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
 }
 

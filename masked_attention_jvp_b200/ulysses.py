@@ -13,9 +13,9 @@ Here the six inputs travel in one all-to-all. The four outputs return one of
 two ways:
   - two all-to-alls (the bf16 pair O, tO and the fp32 pair LSE, tLSE), or
   - with fused_output=True, no collective at all: the kernel's epilogue writes
-    every output row into the symmetric-memory slice buffers of the rank that
-    owns its tokens (caj_attn_fwd_jvp_scatter), over NVLink, and two
-    stream-ordered barriers fence the writes.
+    every output row into the slice buffer of the rank that owns its tokens
+    (caj_attn_fwd_jvp_scatter), mapped from that rank by CUDA IPC, over NVLink,
+    and two stream-ordered barriers (caj_signal_barrier) fence the writes.
 The mask needs no translation, because the local call sees the whole packed
 sequence. Collectives go through torch.distributed (NCCL over NVLink on GPUs).
 All arithmetic is in the local kernel.
@@ -65,16 +65,42 @@ def head_to_seq(y: torch.Tensor, group=None) -> torch.Tensor:
     return recv.permute(1, 2, 0, 3, 4, 5).reshape(S, B, P * Hp, Ls, E)
 
 
-class SliceBuffers:
-    """This rank's output slice in symmetric memory, mapped on every rank.
+class PeerView:
+    """A [shape] view of `dtype` elements at a device address mapped from
+    another rank (an IPC mapping). It offers what attn_fwd_jvp_scatter reads
+    from a slice buffer (shape, dtype, data_ptr) and nothing else: peer memory
+    is written by the scattering kernel, never through PyTorch here."""
 
-    One allocation holds O, tO [B, H, Ls, D], LSE, tLSE [B, H, Ls] fp32 and a
-    pad of signal words for the barrier (regions 256-byte aligned). o[r],
-    to[r], lse[r], tlse[r] view rank r's copy: rank r's device memory, reached
-    over NVLink for r != this rank."""
+    is_cuda = True
+
+    def __init__(self, address: int, shape, dtype: torch.dtype):
+        self._address = int(address)
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+
+    def data_ptr(self) -> int:
+        return self._address
+
+    def dim(self) -> int:
+        return len(self.shape)
+
+    def is_contiguous(self) -> bool:
+        return True
+
+
+class SliceBuffers:
+    """This rank's output slice, mapped by every rank of the group.
+
+    One device allocation holds O, tO [B, H, Ls, D], LSE, tLSE [B, H, Ls] fp32
+    and a pad of signal words for the barrier (regions 256-byte aligned). The
+    ranks swap CUDA IPC handles of their allocations (one all_gather_object)
+    and each maps the others' as plain peer memory: no multicast object is
+    created or bound. o[r], to[r], lse[r], tlse[r] are rank r's slice: this
+    rank's own tensors for r == rank, PeerView mappings reached over NVLink
+    for the others."""
 
     def __init__(self, B: int, H: int, Ls: int, D: int, dtype: torch.dtype, device, group=None):
-        import torch.distributed._symmetric_memory as symm_mem
+        from . import ipc_export, ipc_open
 
         def up(x):
             return (x + 255) // 256 * 256
@@ -85,24 +111,37 @@ class SliceBuffers:
         pad_off = offs[3] + up(n_st * 4)
         total = pad_off + 256
         self.key = (B, H, Ls, D, dtype, torch.device(device))
-        self.buf = symm_mem.empty(total, dtype=torch.uint8, device=device)
-        # the signal pad starts at zero before any peer can reach it: the
-        # rendezvous below is the first point where peers learn its address
-        self.buf.zero_()
+        self.rank, self.world = dist.get_rank(group), dist.get_world_size(group)
+        # zeroed (the signal pad included) before any peer can learn its address
+        self.buf = torch.zeros(total, dtype=torch.uint8, device=device)
         torch.cuda.synchronize(device)
-        self.handle = symm_mem.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
-        self.rank, self.world = self.handle.rank, self.handle.world_size
-        hd = self.handle
+        handles = [None] * self.world
+        dist.all_gather_object(handles, ipc_export(self.buf), group=group)
+        self._opened = []
+        bases = []
+        for r in range(self.world):
+            if r == self.rank:
+                bases.append(self.buf.data_ptr())
+            else:
+                addr = ipc_open(handles[r])
+                self._opened.append(addr)
+                bases.append(addr)
+        me = self.rank
 
         def view(r, off, shape, dt):
-            return hd.get_buffer(r, shape, dt, off // torch.empty((), dtype=dt).element_size())
+            if r == me:
+                n = 1
+                for x in shape:
+                    n *= x
+                return self.buf[off:off + n * torch.empty((), dtype=dt).element_size()].view(dt).view(shape)
+            return PeerView(bases[r] + off, shape, dt)
 
         P = self.world
         self.o = [view(r, offs[0], (B, H, Ls, D), dtype) for r in range(P)]
         self.to = [view(r, offs[1], (B, H, Ls, D), dtype) for r in range(P)]
         self.lse = [view(r, offs[2], (B, H, Ls), torch.float32) for r in range(P)]
         self.tlse = [view(r, offs[3], (B, H, Ls), torch.float32) for r in range(P)]
-        self.pads = [view(r, pad_off, (64,), torch.int32).data_ptr() for r in range(P)]
+        self.pads = [bases[r] + pad_off for r in range(P)]
         self.epoch = 0
 
     def barrier(self, timeout_ms: int = 10000):
@@ -114,6 +153,14 @@ class SliceBuffers:
         from . import signal_barrier
         self.epoch += 1
         signal_barrier(self.pads, self.rank, self.epoch, timeout_ms)
+
+    def close(self):
+        """Unmaps the peers' slices (after this rank's last use of them)."""
+        from . import ipc_close
+        torch.cuda.synchronize(self.buf.device)
+        for addr in self._opened:
+            ipc_close(addr)
+        self._opened = []
 
 
 class _LocalSlices:
@@ -162,7 +209,7 @@ def ulysses_attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = Non
 
     fused_output=True (CUDA tensors, the fused kernel): the output all-to-all
     is done by the kernel's epilogue, which stores each row into the
-    symmetric-memory slice buffer of its owner (see SliceBuffers). The
+    slice buffer of its owner, mapped by CUDA IPC (see SliceBuffers). The
     returned tensors are copies, so the slice buffers are free for the next
     call once every rank has passed its first barrier. Without a process group
     (a single process) the one slice is ordinary device memory. The barriers
@@ -210,5 +257,10 @@ def _ulysses_fused_output(ins, mask, scale, group, clean_tangent_zero, slices=No
 
 
 def release_slice_buffers() -> None:
-    """Drops the cached slice buffers (before the process group goes away)."""
+    """Unmaps and drops the cached slice buffers (before the process group
+    goes away)."""
+    for sb in _slice_buffers.values():
+        close = getattr(sb, "close", None)
+        if close is not None:
+            close()
     _slice_buffers.clear()

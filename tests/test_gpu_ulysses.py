@@ -1,9 +1,9 @@
 """Ulysses path on the GPU with the real kernel: a one-rank NCCL group (this
 machine gives one GPU per run), so the all-to-alls are identities and the result
 must equal the direct call bit for bit, and the fp64 oracle within the bf16
-tolerances of the parity tests. The fused-output form runs through symmetric
-memory, the library's signal barrier and the scattering kernel on the same
-group, and through ordinary memory without a process group. Multi-rank layout
+tolerances of the parity tests. The fused-output form runs through the IPC
+slice buffers, the library's signal barrier and the scattering kernel on the
+same group, and through ordinary memory without a process group. Multi-rank layout
 and arithmetic are covered by the gloo tests on the CPU, and the scatter over
 several slices by the emulated ranks of test_gpu_scatter."""
 import contextlib

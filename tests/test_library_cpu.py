@@ -358,3 +358,17 @@ def test_signal_barrier_validation_launches_nothing():
     assert call([0x1000, 0x2002], 2, 0, 1) == INV                          # misaligned pad
     if _NO_GPU:
         assert call([0x1000, 0x2000], 2, 1, 7) == _lib.CAJ_ERR_CUDA        # valid: stops at the device check
+
+
+def test_ipc_entry_points_validate_without_a_gpu():
+    L = _lib.lib()
+    INV = _lib.CAJ_ERR_INVALID_ARG
+    h = _lib.IpcHandleC()
+    p = ctypes.c_void_p(0)
+    assert L.caj_ipc_export(None, ctypes.byref(h)) == INV
+    assert L.caj_ipc_export(ctypes.c_void_p(0x1000), None) == INV
+    assert L.caj_ipc_open(None, ctypes.byref(p)) == INV
+    assert L.caj_ipc_open(ctypes.byref(h), None) == INV
+    assert L.caj_ipc_close(ctypes.c_void_p(0x1000)) == INV          # never opened here
+    assert L.caj_ipc_close(None) == INV
+    assert ctypes.sizeof(_lib.IpcHandleC) == 72
