@@ -295,11 +295,13 @@ caj_status caj_attn_fwd_jvp_host_static(const void *q, const void *k, const void
  *        w       [C, K] bf16 row-major (the layer's weight)
  *        bias    [C] bf16, or null for none
  *   out: y, ty   [M, C] bf16, fully overwritten
- * Two bf16 GEMMs with fp32 accumulation (cuBLASLt, bias fused as its
- * epilogue). No workspace: nothing is allocated per call. Pointers 16-byte
- * aligned; K and C multiples of 8 (CAJ_ERR_UNSUPPORTED otherwise). Returns
- * CAJ_OK once enqueued on `stream`, CAJ_ERR_INVALID_ARG without launching,
- * or CAJ_ERR_CUDA (cuBLASLt refused; caj_last_cuda_error names its status).
+ * One launch of a tcgen05 kernel computes both products (the rows of x and tx
+ * form one operand, so each weight tile serves both), bf16 in, fp32
+ * accumulation, the bias added in fp32 to primal rows before the rounding to
+ * bf16. Nothing is allocated per call. Pointers 16-byte aligned; K and C
+ * multiples of 8 and M < 2^31 (CAJ_ERR_UNSUPPORTED otherwise). Returns CAJ_OK
+ * once enqueued on `stream`, CAJ_ERR_INVALID_ARG without launching, or
+ * CAJ_ERR_CUDA. Bounded-wait failures are reported by caj_last_device_status.
  */
 typedef struct {
   int64_t M;

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcausaljvp.so")
 SOURCES = ["api.cpp", "fwd_jvp_sm100.cu", "fwd_jvp_simt.cu", "prologue.cu", "bwd_sm100.cu",
-           "host_static.cu", "signal.cu"]
+           "host_static.cu", "signal.cu", "out_proj_sm100.cu"]
 HEADERS = ["kernels.h", "mask_schedule.h", "ptx_sm100.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -60,7 +60,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
         objs.append(obj)
     tmp = LIB + f".tmp{os.getpid()}"
-    r = subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static", "-lcublasLt"],
+    r = subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"],
                        capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

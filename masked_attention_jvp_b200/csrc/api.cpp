@@ -3,7 +3,6 @@
 // include/causaljvp.h for the contract of every entry point.
 #include "causaljvp.h"
 
-#include <cublasLt.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -124,80 +123,18 @@ uint64_t wait_timeout_ns() {
 
 namespace {
 
-// ------------------------------------------------ output projection (cuBLASLt)
-// y = x W^T (+ bias), ty = tx W^T: two plain bf16 GEMMs with fp32
-// accumulation, the bias fused as cuBLASLt's epilogue. Row-major y[M][C] is the
-// column-major C x M matrix W (C x K) times x^T (K x M): A = w stored K x C
-// (transposed), B = x stored K x M, D = y stored C x M. No workspace, so
-// nothing is allocated per call; the handle is created once per process.
-caj_status lt_fail(cublasStatus_t s) {
-  std::snprintf(g_cuda_msg, sizeof g_cuda_msg, "cublasLt status %d", int(s));
-  return CAJ_ERR_CUDA;
-}
-
-cublasStatus_t lt_handle(cublasLtHandle_t *h) {
-  static std::mutex mu;
-  static cublasLtHandle_t handle = nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!handle) {
-    cublasStatus_t s = cublasLtCreate(&handle);
-    if (s != CUBLAS_STATUS_SUCCESS) return s;
-  }
-  *h = handle;
-  return CUBLAS_STATUS_SUCCESS;
-}
-
-cublasStatus_t lt_gemm(cublasLtHandle_t lt, const void *a_w, const void *b_x, void *d_y,
-                       const void *bias, int64_t M, int64_t K, int64_t C, cudaStream_t s) {
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, ld = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  cublasStatus_t r = cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F);
-  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-  if (r == CUBLAS_STATUS_SUCCESS)
-    r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta));
-  if (r == CUBLAS_STATUS_SUCCESS)
-    r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb));
-  if (r == CUBLAS_STATUS_SUCCESS && bias) {
-    const cublasLtEpilogue_t ep = CUBLASLT_EPILOGUE_BIAS;
-    const cudaDataType_t bt = CUDA_R_16BF;
-    r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_EPILOGUE, &ep, sizeof(ep));
-    if (r == CUBLAS_STATUS_SUCCESS)
-      r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_BIAS_POINTER, &bias, sizeof(bias));
-    if (r == CUBLAS_STATUS_SUCCESS)
-      r = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_BIAS_DATA_TYPE, &bt, sizeof(bt));
-  }
-  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, K, C, K);
-  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, K, M, K);
-  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatrixLayoutCreate(&ld, CUDA_R_16BF, C, M, C);
-  if (r == CUBLAS_STATUS_SUCCESS) r = cublasLtMatmulPreferenceCreate(&pref);
-  const size_t no_workspace = 0;
-  if (r == CUBLAS_STATUS_SUCCESS)
-    r = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &no_workspace,
-                                             sizeof(no_workspace));
-  cublasLtMatmulHeuristicResult_t heur{};
-  int found = 0;
-  if (r == CUBLAS_STATUS_SUCCESS)
-    r = cublasLtMatmulAlgoGetHeuristic(lt, op, la, lb, ld, ld, pref, 1, &heur, &found);
-  if (r == CUBLAS_STATUS_SUCCESS && found == 0) r = CUBLAS_STATUS_NOT_SUPPORTED;
-  const float one = 1.f, zero = 0.f;
-  if (r == CUBLAS_STATUS_SUCCESS)
-    r = cublasLtMatmul(lt, op, &one, a_w, la, b_x, lb, &zero, d_y, ld, d_y, ld, &heur.algo, nullptr, 0, s);
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (ld) cublasLtMatrixLayoutDestroy(ld);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return r;
-}
-
-caj_status out_proj_gemms(const void *x, const void *tx, const void *w, const void *bias, int64_t M,
-                          int64_t K, int64_t C, void *y, void *ty, cudaStream_t s) {
-  cublasLtHandle_t lt = nullptr;
-  cublasStatus_t r = lt_handle(&lt);
-  if (r == CUBLAS_STATUS_SUCCESS) r = lt_gemm(lt, w, x, y, bias, M, K, C, s);        // primal
-  if (r == CUBLAS_STATUS_SUCCESS) r = lt_gemm(lt, w, tx, ty, nullptr, M, K, C, s);   // tangent
-  return r == CUBLAS_STATUS_SUCCESS ? CAJ_OK : lt_fail(r);
+// ------------------------------------------------ output projection
+// 2-D bf16 map over a row-major [rows, cols] matrix, box = 64 columns x box_rows,
+// 128-byte swizzle, zero fill outside the matrix.
+bool encode_map_2d(EncodeTiledFn enc, CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
+                   int box_rows) {
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Shape, dtype, flag and mask checks shared by the device and host forms of
@@ -610,10 +547,25 @@ caj_status caj_out_proj_jvp(const void *x, const void *tx, const void *w, const 
   for (const void *p : ptrs)
     if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
   if (bias && !aligned16(bias)) return CAJ_ERR_INVALID_ARG;
+  if (shape->M > (int64_t(1) << 31) - 1) return CAJ_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
   caj_status st = check_device();
   if (st != CAJ_OK) return st;
-  return out_proj_gemms(x, tx, w, bias, shape->M, shape->K, shape->C, y, ty,
-                        static_cast<cudaStream_t>(stream));
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+  caj::OutProjParams p{};
+  const int64_t M = shape->M, K = shape->K, C = shape->C;
+  const bool okm = encode_map_2d(enc, &p.tm_x, x, M, K, 128) && encode_map_2d(enc, &p.tm_tx, tx, M, K, 128) &&
+                   encode_map_2d(enc, &p.tm_w, w, C, K, 128) && encode_map_2d(enc, &p.tm_y, y, M, C, 32) &&
+                   encode_map_2d(enc, &p.tm_ty, ty, M, C, 32);
+  if (!okm) return cuda_fail(cudaErrorInvalidValue);
+  p.bias = bias;
+  p.M = int32_t(M);
+  p.K = K;
+  p.C = C;
+  p.timeout_ns = wait_timeout_ns();
+  p.fault_mode = g_fault_mode.load();
+  cudaError_t e = caj::launch_out_proj_sm100(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
 }
 
 caj_status caj_qk_norm_rope_jvp(const void *xq, const void *xk, const void *xv, const void *txq,
@@ -800,8 +752,12 @@ caj_status caj_last_device_status(void *stream) {
   if (e != cudaSuccess) return cuda_fail(e);
   e = caj::read_and_clear_signal_error(&scode);
   if (e != cudaSuccess) return cuda_fail(e);
+  uint32_t pcode = 0;
+  e = caj::read_and_clear_proj_error(&pcode);
+  if (e != cudaSuccess) return cuda_fail(e);
   if (!code) code = bcode;
   if (!code) code = scode;
+  if (!code) code = pcode;
   if (code != 0) {
     g_last_device_code = code;
     return CAJ_ERR_DEVICE_TIMEOUT;

@@ -143,6 +143,19 @@ struct BwdParams {
   int32_t fault_mode;     // test hook: 1 = the producers issue no copies
 };
 
+// Output projection in primal-tangent form: y = x W^T + b, ty = tx W^T.
+// 2-D bf16 maps, innermost dimension first, 128-byte swizzle:
+//   tm_x, tm_tx over [M, K], box 64 x 128 (a CTA's half of a 256-row tile);
+//   tm_w over [C, K], box 64 x 128 (a CTA's half of a 256-row weight tile);
+//   tm_y, tm_ty over [M, C], box 64 x 32 (the epilogue's store box).
+struct OutProjParams {
+  CUtensorMap tm_x, tm_tx, tm_w, tm_y, tm_ty;
+  const void *bias;      // [C] bf16 or null
+  int32_t M, K, C;
+  uint64_t timeout_ns;
+  int32_t fault_mode;    // test hook: 1 = the producer issues no copies
+};
+
 // Signal barrier of a context-parallel group: pads[r] is rank r's pad of
 // kMaxShards words as mapped in this process.
 struct SignalParams {
@@ -159,6 +172,8 @@ cudaError_t launch_qk_norm_rope_jvp(const PrologueParams &p, cudaStream_t stream
 cudaError_t launch_attn_bwd_sm100(const BwdParams &p, int D, cudaStream_t stream);
 cudaError_t read_and_clear_bwd_error(uint32_t *out);
 cudaError_t launch_signal_barrier(const SignalParams &p, cudaStream_t stream);
+cudaError_t launch_out_proj_sm100(const OutProjParams &p, cudaStream_t stream);
+cudaError_t read_and_clear_proj_error(uint32_t *out);
 cudaError_t read_and_clear_signal_error(uint32_t *out);
 
 // Device error word access (defined next to the kernels that write it).

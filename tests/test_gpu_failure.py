@@ -108,3 +108,32 @@ def test_backward_kernels_time_out_too():
     assert rel(dq.float().cpu().numpy(), rq) <= 2e-2
     assert rel(dk.float().cpu().numpy(), rk) <= 2e-2
     assert rel(dv.float().cpu().numpy(), rv) <= 1e-2
+
+
+def test_output_projection_times_out_too():
+    """The projection kernel bounds its waits the same way: with the hook its
+    producer issues no copies, the MMA thread's first wait runs out, and the
+    next normal call is correct."""
+    L = _lib.lib()
+    g = torch.Generator(device="cuda").manual_seed(12)
+    x, tx = (torch.randn(256, 128, device="cuda", generator=g).to(torch.bfloat16) for _ in range(2))
+    wt = (torch.randn(256, 128, device="cuda", generator=g) / 128 ** 0.5).to(torch.bfloat16)
+    caj.device_status()
+    assert L.caj_set_wait_timeout_ms(100.0) == _lib.CAJ_OK
+    assert L.caj_debug_set_fault(1) == _lib.CAJ_OK
+    try:
+        caj.out_proj_jvp(x, tx, wt)
+        with pytest.raises(caj.CajError) as err:
+            caj.device_status()
+        assert err.value.status == _lib.CAJ_ERR_DEVICE_TIMEOUT
+        assert L.caj_last_device_error_code() & 0xFF00 == 0x100
+    finally:
+        L.caj_debug_set_fault(0)
+        L.caj_set_wait_timeout_ms(0.0)
+    caj.device_status()
+    y, ty = caj.out_proj_jvp(x, tx, wt)
+    caj.device_status()
+    ry, rty = oracle.out_proj_jvp(x, tx, wt)
+    rel = lambda a, b: float(np.linalg.norm(a - b) / np.linalg.norm(b))
+    assert rel(y.float().cpu().numpy(), ry) <= 1e-2
+    assert rel(ty.float().cpu().numpy(), rty) <= 1e-2

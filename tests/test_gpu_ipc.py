@@ -8,6 +8,7 @@ IPC mapping into A's memory, which is what a peer rank's slice is on a
 multi-GPU run. The processes meet only on the host (a queue), never through a
 GPU wait. A then checks its slice against its own direct call, bit for bit,
 and against the fp64 oracle."""
+import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
@@ -42,7 +43,10 @@ def _writer(handles, q):
         caj2.device_status()
         for a in addrs:
             caj2.ipc_close(a)
-        q.put(("ok", [t.cpu() for t in mine]))
+        # plain numpy arrays: torch tensors would travel as file descriptors that
+        # this process must outlive
+        q.put(("ok", [t.cpu().view(torch.int16).numpy() if t.dtype == torch.bfloat16 else t.cpu().numpy()
+                      for t in mine]))
     except BaseException as e:  # report, never hang the parent
         q.put(("error", repr(e)))
 
@@ -63,6 +67,8 @@ def test_ipc_mapped_slice_receives_the_scattered_rows():
     p.join(timeout=60)
     assert status == "ok", payload
     assert p.exitcode == 0
+    payload = [torch.from_numpy(a).view(torch.bfloat16) if a.dtype == np.int16 else torch.from_numpy(a)
+               for a in payload]
     torch.cuda.synchronize()
     ins = make_inputs(W, "cuda")
     direct = caj.attn_fwd_jvp(*ins, W.mask)

@@ -45,7 +45,10 @@ def test_token_major_output_is_the_head_major_output_permuted(case):
 
 
 @pytest.mark.parametrize("M,K,C,with_bias", [(37, 64, 72, True), (1000, 1536, 1536, True),
-                                             (4096, 1536, 1536, False), (1, 128, 8, True)])
+                                             (4096, 1536, 1536, False), (1, 128, 8, True),
+                                             (300, 200, 520, True),     # ragged K block, partial column box
+                                             (2000, 40, 1032, False),   # K below one stage, 5 column blocks
+                                             (129, 5120, 64, True)])    # long K, one column box
 def test_out_proj_matches_oracle(M, K, C, with_bias):
     g = torch.Generator(device="cuda").manual_seed(M + K + C)
     x, tx = (torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16) for _ in range(2))
@@ -58,6 +61,45 @@ def test_out_proj_matches_oracle(M, K, C, with_bias):
         got = got.float().cpu().numpy()
         assert rel_fro(got, ref) <= 1e-2
         assert float(np.max(np.abs(got - ref))) <= 1e-2 * float(np.max(np.abs(ref)))
+
+
+def test_out_proj_full_size_rows_match_oracle():
+    """The bench's shape: the TF frame-wise workload's tokens (M = 65520, which
+    is not a multiple of the 128-row tile), K = C = 1536. Rows sampled across
+    the whole range, the last row block of x and of tx included."""
+    M, K, C = 65520, 1536, 1536
+    g = torch.Generator(device="cuda").manual_seed(9)
+    x, tx = (torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16) for _ in range(2))
+    wt = (torch.randn(C, K, device="cuda", generator=g) / K ** 0.5).to(torch.bfloat16)
+    b = torch.randn(C, device="cuda", generator=g).to(torch.bfloat16)
+    y, ty = caj.out_proj_jvp(x, tx, wt, b)
+    torch.cuda.synchronize()
+    caj.device_status()
+    gen = torch.Generator().manual_seed(10)
+    rows = torch.unique(torch.cat([torch.randint(0, M, (2048,), generator=gen), torch.arange(M - 200, M),
+                                   torch.arange(0, 130)]))
+    idx = rows.cuda()
+    ry, rty = oracle.out_proj_jvp(x[idx], tx[idx], wt, b)
+    for got, ref in ((y[idx], ry), (ty[idx], rty)):
+        got = got.float().cpu().numpy()
+        assert rel_fro(got, ref) <= 1e-2
+        assert float(np.max(np.abs(got - ref))) <= 1e-2 * float(np.max(np.abs(ref)))
+
+
+def test_out_proj_writes_nothing_past_its_rows_and_columns():
+    """Output rows and columns outside [M, C] stay untouched (the tile store
+    clips them): a larger buffer around y keeps its sentinel values."""
+    M, K, C = 150, 64, 72
+    g = torch.Generator(device="cuda").manual_seed(11)
+    x, tx = (torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16) for _ in range(2))
+    wt = (torch.randn(C, K, device="cuda", generator=g) / K ** 0.5).to(torch.bfloat16)
+    big = torch.full((M + 64, C), 7.0, dtype=torch.bfloat16, device="cuda")
+    bigt = torch.full((M + 64, C), 7.0, dtype=torch.bfloat16, device="cuda")
+    caj.out_proj_jvp(x, tx, wt, None, out=(big[:M], bigt[:M]))
+    torch.cuda.synchronize()
+    assert torch.all(big[M:] == 7.0) and torch.all(bigt[M:] == 7.0)
+    ry, rty = oracle.out_proj_jvp(x, tx, wt, None)
+    assert rel_fro(big[:M].float().cpu().numpy(), ry) <= 1e-2
 
 
 def test_attention_then_projection_chain():
