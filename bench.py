@@ -9,11 +9,13 @@ single-GPU run also times the other four workloads (one key each under
 clean-tangent-zero call and the context-parallel scatter.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--split heads|replicas|ulysses] [--fused-output]
+                    [--split tiles|heads|replicas|ulysses] [--fused-output]
 
 Prints one JSON line on rank 0. Multi-GPU runs (torchrun) split one problem:
-by default its heads go to the ranks (independent problems, no data-path
-collective, strong scaling); --split ulysses gives every rank a sequence shard
+by default its 128-row query tiles are dealt out to the ranks by cost, every
+rank holding the whole inputs and running its tiles for every head
+(independent problems, no data-path collective, strong scaling); --split heads
+gives every rank whole heads; --split ulysses gives every rank a sequence shard
 and runs the Ulysses all-to-all path; --split replicas gives every rank its own
 copy (weak scaling). Throughput is whole-job work over the slowest rank's time.
 """
@@ -47,9 +49,12 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 KERNEL_SOURCES = ["fwd_jvp_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct Sm100Params"]
 PROLOGUE_SOURCES = ["prologue.cu", "struct PrologueParams"]
 BACKWARD_SOURCES = ["bwd_sm100.cu", "ptx_sm100.cuh", "mask_schedule.h", "struct BwdParams"]
+OUT_PROJ_SOURCES = ["out_proj_sm100.cu", "ptx_sm100.cuh", "struct OutProjParams"]
 # {(workload, code hash of the kernel's sources): dram bytes read + written per launch}
 MEASURED_TRAFFIC = {("wan1.3b_tf_framewise", "2eecf04220eab7c1"): 1431131648 + 390999296}
 PROLOGUE_TRAFFIC = {("wan1.3b_tf_framewise", "34494554b0571872"): 1241276160 + 1150380544}
+# one launch of the output projection on the workload's tokens (M = 65520, K = C = 1536)
+OUT_PROJ_TRAFFIC = {("wan1.3b_tf_framewise", "8b4c659bc7ef9add"): 407464960 + 368277760}
 # summed over the three launches of one backward call (delta, dQ, dK/dV)
 BACKWARD_TRAFFIC = {("wan1.3b_tf_framewise", "eb90badc0d3e064a"):
                     402579712 + 8373760 + 814591488 + 183904256 + 817019904 + 383885056}
@@ -468,6 +473,8 @@ def bench_out_proj(w, dev, steps, peaks):
     return {"op": "y = x W^T + b, ty = tx W^T (out_proj_sm100_kernel, one launch)", "M": M, "K": K, "C": C,
             "ms": round(ms, 4), "bound": "tensor", "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(tf / peak, 4), "kernel": "out_proj_sm100_kernel",
+            "traffic": OUT_PROJ_TRAFFIC.get((w.name, kernel_sources_hash(OUT_PROJ_SOURCES))),
+            "algorithmic_bytes": 2 * (2 * M * K + K * C + 2 * M * C) + 2 * C,
             "cublas_reference": {"ms": round(ms_lib, 4), "tflops": round(fl / (ms_lib / 1e3) / 1e12, 2),
                                  "what": "torch.addmm + torch.mm (cuBLAS) on the same tensors"},
             "timing": "best of 2 alternating rounds of %d calls each" % steps}
@@ -621,11 +628,50 @@ def bench_e2e(args, w, host, fl_job, world, stream, dev, barrier):
             "api": "attn_fwd_jvp on pinned CPU tensors (caj_attn_fwd_jvp_host)"}
 
 
+def bench_e2e_part(args, w, host, fl_job, world, rank, stream, dev, barrier):
+    """The e2e leg of the query-tile split: every step each rank copies the
+    whole inputs from pinned host memory, runs its part through the public
+    API (attn_fwd_jvp_out with part=(rank, world)) and copies the four output
+    buffers back to pinned host memory, all on one stream."""
+    import masked_attention_jvp_b200 as caj
+    pinned = [t.pin_memory() for t in host]
+    dins = [torch.empty_like(t, device=dev) for t in pinned]
+    o, to = torch.empty_like(dins[0]), torch.empty_like(dins[0])
+    lse = torch.empty(dins[0].shape[:3], dtype=torch.float32, device=dev)
+    tlse = torch.empty_like(lse)
+    hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, to, lse, tlse)]
+    h2d = sum(t.numel() * t.element_size() for t in pinned)
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+
+    def step():
+        for d, h in zip(dins, pinned):
+            d.copy_(h, non_blocking=True)
+        caj.attn_fwd_jvp_out(*dins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream, part=(rank, world))
+        for h, d in zip(hout, (o, to, lse, tlse)):
+            h.copy_(d, non_blocking=True)
+
+    step()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(strong_tflops(fl_job, args.steps, ms), 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.steps,
+            "ms_per_step": round(ms / args.steps, 3), "clocks": clk.summary(),
+            "api": "attn_fwd_jvp_out(part=(rank, world)) between pinned-host copies, per rank"}
+
+
 def rank_inputs(args, w, host, world, rank):
     """This rank's share of the workload's inputs (host tensors) and the
     problem it runs, by the split mode."""
-    if world == 1 or args.split == "replicas":
-        return host, w
+    if world == 1 or args.split in ("replicas", "tiles"):
+        return host, w  # tiles: every rank holds the whole inputs and runs its part of the query tiles
     if args.split == "heads":
         h0, h1 = split_heads(w.H, world, rank)
         return [t[:, h0:h1].contiguous() for t in host], w
@@ -666,10 +712,12 @@ def bench_gpu(args, rank, world, local_rank):
         lse = torch.empty(ins[0].shape[:3], dtype=torch.float32, device=dev)
         tlse = torch.empty_like(lse)
 
+        part = (rank, world) if (args.split == "tiles" and world > 1) else None
+
         def step():
             if have_work:
                 caj.attn_fwd_jvp_out(*ins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream,
-                                     clean_tangent_zero=args.clean_tangent_zero)
+                                     clean_tangent_zero=args.clean_tangent_zero, part=part)
         L = w.mask.n_frames * w.mask.tokens_per_frame
         launches_per_step = (2 if args.clean_tangent_zero and L >= 128 else 1) if have_work else 0
 
@@ -700,8 +748,10 @@ def bench_gpu(args, rank, world, local_rank):
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e and args.split != "ulysses":
+    if not args.no_e2e and (world == 1 or args.split in ("heads", "replicas")):
         e2e = bench_e2e(args, w, host, fl_job, world, stream, dev, barrier)
+    elif not args.no_e2e and args.split == "tiles":
+        e2e = bench_e2e_part(args, w, host, fl_job, world, rank, stream, dev, barrier)
     if rank != 0:
         return None
     peaks, src = load_peaks()
@@ -710,9 +760,11 @@ def bench_gpu(args, rank, world, local_rank):
     kernel_ms = statistics.mean(per)
     rank0_flops = fl if (world == 1 or args.split == "replicas") else fl * (
         (split_heads(w.H, world, 0)[1] - split_heads(w.H, world, 0)[0]) / w.H if args.split == "heads" else 1.0 / world)
+    # (tiles: the parts are balanced to within one query tile's work, so rank 0 does ~1/world)
     achieved = rank0_flops / (kernel_ms / 1e3) / 1e12
     clocks = clk.summary()
-    parallelism = {"heads": f"head split over {world} GPUs", "replicas": f"replica x{world}",
+    parallelism = {"tiles": f"query tiles dealt over {world} GPUs by cost (every head)",
+                   "heads": f"head split over {world} GPUs", "replicas": f"replica x{world}",
                    "ulysses": f"Ulysses context parallelism over {world} GPUs"
                               + (" (output all-to-all in the epilogue)" if args.fused_output else "")}[args.split]
     line = {
@@ -851,9 +903,10 @@ def main():
                     help="skip the clean-tangent-zero sub-measurement (teacher-forcing workloads)")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip timing the other four workloads (the 'configs' key)")
-    ap.add_argument("--split", default="heads", choices=["heads", "replicas", "ulysses"],
-                    help="multi-GPU work split: the problem's heads over the ranks (default, strong scaling), "
-                         "a copy per rank (weak scaling), or Ulysses sequence shards with all-to-alls")
+    ap.add_argument("--split", default="tiles", choices=["tiles", "heads", "replicas", "ulysses"],
+                    help="multi-GPU work split: the query tiles dealt over the ranks by cost (default, strong "
+                         "scaling), the heads over the ranks, a copy per rank (weak scaling), or Ulysses sequence "
+                         "shards with all-to-alls")
     ap.add_argument("--fused-output", action="store_true",
                     help="with --split ulysses: the output all-to-all in the attention epilogue")
     ap.add_argument("--heads", type=int, default=None,

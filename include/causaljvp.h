@@ -115,6 +115,27 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v,
                             void *stream);
 
 /*
+ * One part of caj_attn_fwd_jvp, for splitting one call over `nparts` GPUs with
+ * no collective: every (batch, head) and every query row is an independent
+ * problem (appendix B: each query block runs on its own over the key ranges its
+ * mask allows), so rank r may compute any subset of the query tiles (128 rows)
+ * while holding all of q..tv. The tiles are dealt out by cost, heaviest first,
+ * each to the part with the least work so far, so parts differ by at most one
+ * tile's work; a part runs its tiles for every head.
+ *   in / out     as caj_attn_fwd_jvp (full-size buffers); only the rows of this
+ *                part's query tiles are written, the others are left as they are
+ *   part, nparts 0 <= part < nparts; nparts = 1 is caj_attn_fwd_jvp
+ * The union over parts 0..nparts-1 equals caj_attn_fwd_jvp bit for bit.
+ * bf16 only when nparts > 1 (CAJ_ERR_UNSUPPORTED for fp32). Returns as
+ * caj_attn_fwd_jvp; a part without tiles launches nothing and returns CAJ_OK.
+ */
+caj_status caj_attn_fwd_jvp_part(const void *q, const void *k, const void *v,
+                                 const void *tq, const void *tk, const void *tv,
+                                 const caj_problem *prob, const caj_mask_desc *mask,
+                                 int32_t part, int32_t nparts, void *o, void *to, float *lse,
+                                 float *tlse, void *stream);
+
+/*
  * Context-parallel form of caj_attn_fwd_jvp, with the output all-to-all done by
  * the kernel's epilogue. Causal-rCM trains with flattened Ulysses context
  * parallelism (section 3.2.1, "Parallelism"; section 3.2.2, "JVP Ulysses CP").
@@ -424,6 +445,13 @@ caj_status caj_key_query_ranges(const caj_mask_desc *mask, int32_t key, int32_t 
  * t[0..5]. Returns the number of tiles, or -1 on a bad argument. */
 int32_t caj_ktile_query_tiles(const caj_mask_desc *mask, int32_t k0, int32_t k1,
                               int32_t block_q, int32_t t[6]);
+
+/* The query tiles (of 128 rows) that part `part` of `nparts` runs in
+ * caj_attn_fwd_jvp_part, in launch order (heaviest first): writes up to
+ * `capacity` tile indices to `tiles` (may be NULL) and returns how many the
+ * part has, or -1 on a bad argument. */
+int32_t caj_part_query_tiles(const caj_mask_desc *mask, int32_t part, int32_t nparts, int32_t *tiles,
+                             int32_t capacity);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int32_t caj_version(void);

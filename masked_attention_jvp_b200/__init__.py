@@ -29,7 +29,7 @@ from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
 __all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "signal_barrier",
-           "ipc_export", "ipc_open", "ipc_close", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
+           "ipc_export", "ipc_open", "ipc_close", "part_query_tiles", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
 
@@ -37,6 +37,16 @@ BLOCK_M = 128  # query rows per tile of both kernels
 BLOCK_N = 64   # keys per tile of the tensor-core kernel
 
 _DTYPES = {torch.float32: _lib.CAJ_DTYPE_F32, torch.bfloat16: _lib.CAJ_DTYPE_BF16}
+
+
+def part_query_tiles(mask, part: int, nparts: int):
+    """The 128-row query tiles part `part` of `nparts` runs, heaviest first."""
+    n = _lib.lib().caj_part_query_tiles(ctypes.byref(_lib.mask_c(mask)), int(part), int(nparts), None, 0)
+    if n < 0:
+        raise ValueError("caj_part_query_tiles rejected its arguments")
+    buf = (ctypes.c_int32 * max(n, 1))()
+    _lib.lib().caj_part_query_tiles(ctypes.byref(_lib.mask_c(mask)), int(part), int(nparts), buf, n)
+    return list(buf[:n])
 
 
 def visible_pairs(mask) -> int:
@@ -85,8 +95,12 @@ def _problem(q: torch.Tensor, scale: Optional[float], clean_tangent_zero: bool =
 
 def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optional[float] = None,
                      stream: Optional[torch.cuda.Stream] = None, clean_tangent_zero: bool = False,
-                     token_major_out: bool = False) -> None:
+                     token_major_out: bool = False, part=None) -> None:
     """Writes into caller-provided CUDA tensors o, to [B,H,N,D] and lse, tlse [B,H,N] fp32.
+
+    part: None for the whole call, or (r, n): only the query tiles of part r
+    of n (cost-balanced, every head; caj_attn_fwd_jvp_part), the way n GPUs
+    split one call with no collective. Rows of other parts are left as they are.
 
     clean_tangent_zero: teacher-forcing layout only; the caller guarantees that
     tq, tk, tv are zero on the clean half, and the kernel skips the products
@@ -110,12 +124,18 @@ def attn_fwd_jvp_out(q, k, v, tq, tk, tv, mask, o, to, lse, tlse, scale: Optiona
         raise ValueError("attn_fwd_jvp_out: lse/tlse must be fp32 [B,H,N]")
     s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
     prob = _problem(q, scale, clean_tangent_zero, token_major_out)
-    st = _lib.lib().caj_attn_fwd_jvp(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
-                                     ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)),
-                                     ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(to.data_ptr()),
-                                     ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(tlse.data_ptr()),
-                                     ctypes.c_void_p(s))
-    _lib.check(st)
+    outs = [ctypes.c_void_p(t.data_ptr()) for t in (o, to, lse, tlse)]
+    if part is None:
+        st = _lib.lib().caj_attn_fwd_jvp(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
+                                         ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)), *outs,
+                                         ctypes.c_void_p(s))
+        _lib.check(st)
+    else:
+        r, n = part
+        st = _lib.lib().caj_attn_fwd_jvp_part(*[ctypes.c_void_p(t.data_ptr()) for t in ins],
+                                              ctypes.byref(prob), ctypes.byref(_lib.mask_c(mask)),
+                                              int(r), int(n), *outs, ctypes.c_void_p(s))
+        _lib.check(st, "caj_attn_fwd_jvp_part")
 
 
 def attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale: Optional[float] = None,

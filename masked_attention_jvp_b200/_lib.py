@@ -19,7 +19,7 @@ EXPORTED = [
     "caj_debug_set_fault", "caj_qk_norm_rope_jvp", "caj_key_query_ranges", "caj_ktile_query_tiles",
     "caj_attn_bwd", "caj_attn_fwd_jvp_host_workspace", "caj_attn_fwd_jvp_host", "caj_out_proj_jvp",
     "caj_attn_fwd_jvp_scatter", "caj_attn_fwd_jvp_host_static", "caj_signal_barrier",
-    "caj_ipc_export", "caj_ipc_open", "caj_ipc_close",
+    "caj_ipc_export", "caj_ipc_open", "caj_ipc_close", "caj_attn_fwd_jvp_part", "caj_part_query_tiles",
 ]
 
 
@@ -133,6 +133,11 @@ def lib() -> ctypes.CDLL:
         L.caj_ipc_open.restype = ctypes.c_int
         L.caj_ipc_close.argtypes = [vp]
         L.caj_ipc_close.restype = ctypes.c_int
+        L.caj_attn_fwd_jvp_part.argtypes = [vp] * 6 + [ctypes.POINTER(ProblemC), ctypes.POINTER(MaskDescC),
+                                                 i32, i32] + [vp] * 5
+        L.caj_attn_fwd_jvp_part.restype = ctypes.c_int
+        L.caj_part_query_tiles.argtypes = [ctypes.POINTER(MaskDescC), i32, i32, ctypes.POINTER(i32), i32]
+        L.caj_part_query_tiles.restype = i32
         L.caj_version.argtypes = []
         L.caj_version.restype = i32
         _lib = L

@@ -288,11 +288,48 @@ int32_t caj_ktile_query_tiles(const caj_mask_desc *mask, int32_t k0, int32_t k1,
 
 namespace {
 
+// The query tiles (of kBlockM rows) in heaviest-first order: by decreasing
+// number of visited key tiles, ties later tile first.
+std::vector<std::pair<int32_t, int32_t>> qtile_costs(const caj::MaskGeom &g) {
+  const int32_t n_qtiles = (g.N + caj::kBlockM - 1) / caj::kBlockM;
+  std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
+  for (int32_t t = 0; t < n_qtiles; ++t) {
+    int32_t r[4];
+    const int32_t q0 = t * caj::kBlockM, q1 = std::min(q0 + caj::kBlockM, g.N);
+    cost[t] = {caj::qtile_key_tiles(g, q0, q1, caj::kBlockN, r[0], r[1], r[2], r[3]), t};
+  }
+  std::sort(cost.begin(), cost.end(), [](const auto &a, const auto &b) {
+    return a.first != b.first ? a.first > b.first : a.second > b.second;
+  });
+  return cost;
+}
+
+// Part `part` of `nparts` of the query tiles, balanced by cost: the tiles go
+// heaviest first, each to the part with the least work so far (lowest index on
+// ties), so parts differ by at most one tile's work. Every head has the same
+// mask, so a part runs its tiles for all heads. Heaviest-first order is kept.
+std::vector<std::pair<int32_t, int32_t>> part_of(const std::vector<std::pair<int32_t, int32_t>> &cost,
+                                                 int32_t part, int32_t nparts) {
+  if (nparts <= 1) return cost;
+  std::vector<int64_t> load(nparts, 0);
+  std::vector<std::pair<int32_t, int32_t>> mine;
+  for (const auto &c : cost) {
+    int32_t best = 0;
+    for (int32_t r = 1; r < nparts; ++r)
+      if (load[r] < load[best]) best = r;
+    load[best] += c.first;
+    if (best == part) mine.push_back(c);
+  }
+  return mine;
+}
+
 // Launches the forward + JVP of a validated problem on `s`, the output rows
 // placed by `out`: a one-slice output, or (scatter) the slices of a
-// context-parallel output.
+// context-parallel output. With nparts > 1 only the query tiles of part
+// `part` run (tensor-core path).
 caj_status fwd_launch(const void *const in[6], const caj_problem *prob, const caj::MaskGeom &g,
-                      const caj::OutMap &out, bool scatter, cudaStream_t s) {
+                      const caj::OutMap &out, bool scatter, cudaStream_t s, int32_t part = 0,
+                      int32_t nparts = 1) {
   const void *q = in[0], *k = in[1], *v = in[2], *tq = in[3], *tk = in[4], *tv = in[5];
   const int64_t BH = int64_t(prob->B) * prob->H;
   const float scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt(float(prob->D));
@@ -337,23 +374,18 @@ caj_status fwd_launch(const void *const in[6], const caj_problem *prob, const ca
   p.timeout_ns = wait_timeout_ns();
   p.fault_mode = g_fault_mode.load();
   p.tile_kind = caj::kTilesAll;
-  // Launch order: query tiles by decreasing number of key tiles (ties: later first).
-  std::vector<std::pair<int32_t, int32_t>> cost(n_qtiles);
-  for (int32_t t = 0; t < n_qtiles; ++t) {
-    int32_t r[4];
-    const int32_t q0 = t * caj::kBlockM, q1 = std::min(q0 + caj::kBlockM, N);
-    cost[t] = {caj::qtile_key_tiles(g, q0, q1, caj::kBlockN, r[0], r[1], r[2], r[3]), t};
-  }
-  std::sort(cost.begin(), cost.end(), [](const auto &a, const auto &b) {
-    return a.first != b.first ? a.first > b.first : a.second > b.second;
-  });
+  // Launch order: query tiles by decreasing number of key tiles (ties: later
+  // first); with parts, this part's tiles only.
+  const std::vector<std::pair<int32_t, int32_t>> cost = part_of(qtile_costs(g), part, nparts);
+  if (cost.empty()) return CAJ_OK;  // a part with no tile: nothing to launch
+  p.n_qtiles = int32_t(cost.size());
   if (prob->flags & CAJ_FLAG_CLEAN_TANGENT_ZERO) {
     // Two launches, each over one kind of query tile in the same heaviest-first
     // order: tiles with a noisy row (the dearer ones) first, then the clean ones.
     std::unique_ptr<caj::Sm100Params> hc(new caj::Sm100Params(p));
     int32_t nn = 0, nc = 0;
-    for (int32_t i = 0; i < n_qtiles; ++i) {
-      const int32_t t = cost[i].second;
+    for (const auto &c : cost) {
+      const int32_t t = c.second;
       if (std::min((t + 1) * caj::kBlockM, N) <= g.L)
         hc->qtile_order[nc++] = uint16_t(t);
       else
@@ -367,7 +399,7 @@ caj_status fwd_launch(const void *const in[6], const caj_problem *prob, const ca
     if (e == cudaSuccess && nc) e = caj::launch_fwd_jvp_sm100(*hc, D, s);
     return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
   }
-  for (int32_t i = 0; i < n_qtiles; ++i) p.qtile_order[i] = uint16_t(cost[i].second);
+  for (size_t i = 0; i < cost.size(); ++i) p.qtile_order[i] = uint16_t(cost[i].second);
 
   cudaError_t e = caj::launch_fwd_jvp_sm100(p, D, s);
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);
@@ -398,6 +430,42 @@ caj_status caj_attn_fwd_jvp(const void *q, const void *k, const void *v, const v
   out.head_base = 0;
   out.token_major = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? 1 : 0;
   return fwd_launch(ins, prob, g, out, false, static_cast<cudaStream_t>(stream));
+}
+
+caj_status caj_attn_fwd_jvp_part(const void *q, const void *k, const void *v, const void *tq,
+                                 const void *tk, const void *tv, const caj_problem *prob,
+                                 const caj_mask_desc *mask, int32_t part, int32_t nparts, void *o,
+                                 void *to, float *lse, float *tlse, void *stream) {
+  const void *ins[6] = {q, k, v, tq, tk, tv};
+  for (const void *p : ins)
+    if (!p || !aligned16(p)) return CAJ_ERR_INVALID_ARG;
+  if (!o || !to || !aligned16(o) || !aligned16(to)) return CAJ_ERR_INVALID_ARG;
+  if (!lse || !tlse || !aligned4(lse) || !aligned4(tlse)) return CAJ_ERR_INVALID_ARG;
+  if (nparts < 1 || part < 0 || part >= nparts) return CAJ_ERR_INVALID_ARG;
+  caj::MaskGeom g;
+  caj_status st = validate_fwd(prob, mask, &g);
+  if (st != CAJ_OK) return st;
+  if (prob->dtype != CAJ_DTYPE_BF16 && nparts > 1) return CAJ_ERR_UNSUPPORTED;  // tensor-core path only
+  st = check_device();
+  if (st != CAJ_OK) return st;
+  caj::OutMap out{};
+  out.o[0] = o; out.to[0] = to; out.lse[0] = lse; out.tlse[0] = tlse;
+  out.shards = 1;
+  out.shard_len = prob->N;
+  out.heads = out.heads_total = prob->H;
+  out.head_base = 0;
+  out.token_major = (prob->flags & CAJ_FLAG_TOKEN_MAJOR_OUT) ? 1 : 0;
+  return fwd_launch(ins, prob, g, out, false, static_cast<cudaStream_t>(stream), part, nparts);
+}
+
+int32_t caj_part_query_tiles(const caj_mask_desc *mask, int32_t part, int32_t nparts, int32_t *tiles,
+                             int32_t capacity) {
+  caj::MaskGeom g;
+  if (!geom_from_desc(mask, &g) || nparts < 1 || part < 0 || part >= nparts || capacity < 0) return -1;
+  const auto mine = part_of(qtile_costs(g), part, nparts);
+  if (tiles)
+    for (size_t i = 0; i < mine.size() && int32_t(i) < capacity; ++i) tiles[i] = mine[i].second;
+  return int32_t(mine.size());
 }
 
 static_assert(CAJ_MAX_SHARDS == caj::kMaxShards, "slice count of the public and kernel output maps");

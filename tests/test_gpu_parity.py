@@ -295,3 +295,39 @@ def test_clean_tangent_zero_repeated_calls_are_bitwise_identical():
         for x, y in zip(first, again):
             assert torch.equal(x, y)
     caj.device_status()
+
+
+PART_CASES = [(MaskDesc(100, 1, 5, 0), 1, 2, 128, False, False), (MaskDesc(37, 1, 7, 1), 2, 2, 128, False, False),
+              (MaskDesc(64, 3, 6, 1), 1, 3, 128, True, False), (MaskDesc(40, 1, 5, 1), 1, 2, 64, False, True),
+              (MaskDesc(5, 1, 3, 1), 1, 2, 128, False, False)]
+
+
+@pytest.mark.parametrize("case", range(len(PART_CASES)))
+@pytest.mark.parametrize("nparts", [2, 3, 8])
+def test_parts_together_equal_the_whole_call(case, nparts):
+    """caj_attn_fwd_jvp_part: run part by part into buffers pre-filled with NaN,
+    the parts write every row exactly as the whole call does (bit for bit),
+    and a part alone leaves the other parts' rows untouched."""
+    from masked_attention_jvp_b200.workloads import zero_clean_tangents
+    mask, B, H, D, ctz, tm = PART_CASES[case]
+    w = Workload(f"part{case}", B, H, D, mask, torch.bfloat16, seed=700 + case, std_tangent=0.5)
+    ins = make_inputs(w, "cuda")
+    if ctz:
+        zero_clean_tangents(w, *ins[3:])
+    whole = caj.attn_fwd_jvp(*ins, w.mask, clean_tangent_zero=ctz, token_major_out=tm)
+    shape = whole[0].shape
+    outs = [torch.full(shape, float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(2)] + \
+        [torch.full(whole[2].shape, float("nan"), device="cuda") for _ in range(2)]
+    for r in range(nparts):
+        caj.attn_fwd_jvp_out(*ins, w.mask, *outs, clean_tangent_zero=ctz, token_major_out=tm, part=(r, nparts))
+        if r == 0:  # part 0 alone wrote its tiles' rows and nothing else
+            torch.cuda.synchronize()
+            rows = torch.zeros(w.N, dtype=torch.bool)
+            for t in caj.part_query_tiles(w.mask, 0, nparts):
+                rows[128 * t:min(128 * t + 128, w.N)] = True
+            lse0 = outs[2].cpu()
+            assert torch.isfinite(lse0[:, :, rows]).all() and torch.isnan(lse0[:, :, ~rows]).all()
+    torch.cuda.synchronize()
+    caj.device_status()
+    for got, want in zip(outs, whole):
+        assert torch.equal(got, want)

@@ -372,3 +372,45 @@ def test_ipc_entry_points_validate_without_a_gpu():
     assert L.caj_ipc_close(ctypes.c_void_p(0x1000)) == INV          # never opened here
     assert L.caj_ipc_close(None) == INV
     assert ctypes.sizeof(_lib.IpcHandleC) == 72
+
+
+@pytest.mark.parametrize("mask", [MaskDesc(1560, 1, 21, 1), MaskDesc(1560, 3, 21, 1), MaskDesc(3600, 1, 21, 0),
+                                  MaskDesc(37, 1, 7, 1), MaskDesc(5, 1, 3, 1)])
+def test_parts_deal_every_query_tile_once_and_balance_the_work(mask):
+    """caj_part_query_tiles: the parts of one call cover every 128-row query
+    tile exactly once, each part's work (visited key tiles) is within one
+    tile's work of every other part's, and each part is in heaviest-first
+    order; one part is the whole call."""
+    N = mask.seq_len
+    n_tiles = (N + 127) // 128
+    cost = {t: caj.qtile_key_tiles(mask, 128 * t, min(128 * t + 128, N))[0] for t in range(n_tiles)}
+    whole = caj.part_query_tiles(mask, 0, 1)
+    assert sorted(whole) == list(range(n_tiles))
+    for nparts in (2, 3, 4, 8):
+        parts = [caj.part_query_tiles(mask, r, nparts) for r in range(nparts)]
+        assert sorted(t for p in parts for t in p) == list(range(n_tiles))
+        loads = [sum(cost[t] for t in p) for p in parts]
+        assert max(loads) - min(loads) <= max(cost.values())
+        for p in parts:
+            assert [cost[t] for t in p] == sorted((cost[t] for t in p), reverse=True)
+
+
+def test_part_entry_validation_launches_nothing():
+    L = _lib.lib()
+    INV, UNS = _lib.CAJ_ERR_INVALID_ARG, _lib.CAJ_ERR_UNSUPPORTED
+    vp = ctypes.c_void_p
+    mask = _lib.MaskDescC(16, 1, 4, 0)
+
+    def call(part, nparts, dtype=_lib.CAJ_DTYPE_BF16):
+        prob = _lib.ProblemC(1, 2, 64, 64, dtype, 0.0, 0)
+        return L.caj_attn_fwd_jvp_part(*[vp(0x10000)] * 6, ctypes.byref(prob), ctypes.byref(mask), part, nparts,
+                                       vp(0x20000), vp(0x20000), vp(0x30000), vp(0x30000), vp(0))
+
+    assert call(0, 0) == INV
+    assert call(2, 2) == INV
+    assert call(-1, 2) == INV
+    assert call(0, 2, _lib.CAJ_DTYPE_F32) == UNS          # the fp32 path runs whole calls only
+    assert L.caj_part_query_tiles(ctypes.byref(mask), 1, 1, None, 0) == -1
+    assert L.caj_part_query_tiles(None, 0, 1, None, 0) == -1
+    if _NO_GPU:
+        assert call(1, 2) == _lib.CAJ_ERR_CUDA             # valid: stops at the device check

@@ -99,3 +99,18 @@ def test_head_split_covers_every_head_once():
             assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
             sizes = [b - a for a, b in ranges]
             assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 0
+
+
+def test_tile_split_parts_balance_for_the_bench_workload():
+    """The default multi-GPU mode deals C2's 512 query tiles over the ranks by
+    cost: with 8 ranks the slowest part carries at most one tile's work more
+    than an even share, so the ideal speed-up is close to 8 (the head split
+    tops out at 6: 12 heads over 8 GPUs)."""
+    import masked_attention_jvp_b200 as caj
+    from masked_attention_jvp_b200.workloads import WORKLOADS
+    m = WORKLOADS["wan1.3b_tf_framewise"].mask
+    N = m.seq_len
+    cost = [caj.qtile_key_tiles(m, 128 * t, min(128 * t + 128, N))[0] for t in range((N + 127) // 128)]
+    for world in (2, 4, 8):
+        loads = [sum(cost[t] for t in caj.part_query_tiles(m, r, world)) for r in range(world)]
+        assert sum(cost) / max(loads) >= world * 0.99
