@@ -699,20 +699,19 @@ template <int D>
 cudaError_t launch_bwd_impl(const BwdParams &p, cudaStream_t stream) {
   using CQ = BCfg<D, 0>;
   using CK = BCfg<D, 1>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static std::atomic<uint64_t> attr_set{0};
+  cudaError_t e = once_per_device(attr_set, [] {
+    cudaError_t r = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          CQ::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CK::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, CK::SMEM_BYTES);
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   const int64_t rows = int64_t(p.BH) * p.geom.N;
   const int64_t threads = rows * (D / 8);
   bwd_delta_kernel<D><<<unsigned((threads + 255) / 256), 256, 0, stream>>>(p.o, p.dout, p.delta, rows);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(p.n_row_tiles) * unsigned(p.BH);
   bwd_dq_kernel<D><<<grid, kThreads, CQ::SMEM_BYTES, stream>>>(p);

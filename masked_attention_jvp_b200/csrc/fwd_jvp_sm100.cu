@@ -1031,13 +1031,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, bool SCATTER>
 cudaError_t launch_primal_impl(const Sm100Params &p, cudaStream_t stream) {
   using C = PCfg<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_primal_sm100_kernel<D, SCATTER>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(fwd_primal_sm100_kernel<D, SCATTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_BYTES);
+  });
+  if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
   fwd_primal_sm100_kernel<D, SCATTER><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError();
@@ -1046,13 +1045,12 @@ cudaError_t launch_primal_impl(const Sm100Params &p, cudaStream_t stream) {
 template <int D, int KIND, bool SCATTER>
 cudaError_t launch_impl(const Sm100Params &p, cudaStream_t stream) {
   using C = Cfg<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D, KIND, SCATTER>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(fwd_jvp_sm100_kernel<D, KIND, SCATTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_BYTES);
+  });
+  if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(p.n_qtiles) * unsigned(p.BH);
   fwd_jvp_sm100_kernel<D, KIND, SCATTER><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError();

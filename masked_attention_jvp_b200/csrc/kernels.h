@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "mask_schedule.h"
 
 namespace caj {
@@ -164,6 +166,22 @@ struct SignalParams {
   uint32_t epoch;
   uint64_t timeout_ns;
 };
+
+// Runs `set` (a per-device kernel attribute setting, e.g. its shared-memory
+// limit) the first time a call site launches on the current device: function
+// attributes hold per device, so a process that drives several GPUs sets them
+// on each. `done` is the call site's bit set of devices (ordinals below 64).
+template <class F>
+inline cudaError_t once_per_device(std::atomic<uint64_t> &done, F set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load() & bit)) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess && bit) done.fetch_or(bit);
+  return e;
+}
 
 // Each returns the launch's cudaError_t (cudaSuccess when enqueued).
 cudaError_t launch_fwd_jvp_sm100(const Sm100Params &p, int D, cudaStream_t stream);

@@ -422,14 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_out_proj_sm100(const OutProjParams &p, cudaStream_t stream) {
-  int dev = 0, sms = 0;
+  int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(out_proj_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const int64_t m_blocks = (p.M + 2 * PM - 1) / (2 * PM), n_blocks = (p.C + PN - 1) / PN;
-  const int64_t tiles = 2 * m_blocks * n_blocks;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -442,10 +437,23 @@ cudaError_t launch_out_proj_sm100(const OutProjParams &p, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cfg.gridDim = dim3(2);
-  int max_pairs = 0;
-  e = cudaOccupancyMaxActiveClusters(&max_pairs, out_proj_sm100_kernel, &cfg);
+  // Per device, once: the shared-memory limit and how many CTA pairs fit at a
+  // time (the persistent grid).
+  static std::atomic<uint64_t> set_up{0};
+  static std::atomic<int> max_pairs_of[64];
+  e = once_per_device(set_up, [&] {
+    cudaError_t r = cudaFuncSetAttribute(out_proj_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
+    int sms = 0, pairs = 0;
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess) r = cudaOccupancyMaxActiveClusters(&pairs, out_proj_sm100_kernel, &cfg);
+    if (r == cudaSuccess && dev < 64) max_pairs_of[dev].store(pairs >= 1 ? pairs : sms / 2);
+    return r;
+  });
   if (e != cudaSuccess) return e;
-  if (max_pairs < 1) max_pairs = sms / 2;
+  const int max_pairs = dev < 64 ? max_pairs_of[dev].load() : 74;
+  const int64_t m_blocks = (p.M + 2 * PM - 1) / (2 * PM), n_blocks = (p.C + PN - 1) / PN;
+  const int64_t tiles = 2 * m_blocks * n_blocks;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
   cfg.gridDim = dim3(unsigned(2 * pairs));
   e = cudaLaunchKernelEx(&cfg, out_proj_sm100_kernel, p);
