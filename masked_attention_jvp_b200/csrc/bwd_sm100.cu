@@ -381,12 +381,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
           rp[i] = v ? rp[i] : __float_as_uint(dl);
         }
       }
+      // element pairs in packed fp32x2 arithmetic (exponentials scalar)
+      const uint64_t sl2x2 = f2(sl2, sl2), nlse2 = f2(-lse2, -lse2), dl2 = f2(dl, dl);
       uint32_t pk[kCols / 2];
 #pragma unroll
       for (int i = 0; i < kCols / 2; ++i) {
-        const float pa = ex2(fmaf(__uint_as_float(rs[2 * i]), sl2, -lse2));
-        const float pb = ex2(fmaf(__uint_as_float(rs[2 * i + 1]), sl2, -lse2));
-        pk[i] = pack_bf16(pa * (__uint_as_float(rp[2 * i]) - dl), pb * (__uint_as_float(rp[2 * i + 1]) - dl));
+        float xa, xb, da, db;
+        f2_split(fma2(f2(__uint_as_float(rs[2 * i]), __uint_as_float(rs[2 * i + 1])), sl2x2, nlse2), xa, xb);
+        const uint64_t p2 = f2(ex2(xa), ex2(xb));
+        f2_split(mul2(p2, sub2(f2(__uint_as_float(rp[2 * i]), __uint_as_float(rp[2 * i + 1])), dl2)), da, db);
+        pk[i] = pack_bf16(da, db);
       }
       tmem_st_cols(cS, pk);
       tmem_wait_st();
@@ -603,20 +607,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       const float4 *st4 = reinterpret_cast<const float4 *>(sgen + C::OFF_ST + s * C::STAGE +
                                                            2 * C::S_BYTES) + (kCols / 4) * g;
       uint32_t pk[kCols / 2], dk[kCols / 2];
+      // element pairs in packed fp32x2 arithmetic (exponentials scalar)
+      const uint64_t sl2x2 = f2(sl2, sl2);
 #pragma unroll
       for (int i4 = 0; i4 < kCols / 4; ++i4) {
         const float4 l4 = st4[i4], d4 = st4[16 + i4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        const uint64_t nl2[2] = {f2(-l4.x, -l4.y), f2(-l4.z, -l4.w)}, dv2[2] = {f2(d4.x, d4.y), f2(d4.z, d4.w)};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int i = 2 * i4 + h, c0 = 2 * i, c1 = 2 * i + 1;
           // hidden pairs: s = -inf gives p = 0, so dS = 0 whatever dP - Delta is
-          const float pa = ex2(fmaf(__uint_as_float(rs[c0]), sl2, -lv[2 * h]));
-          const float pb = ex2(fmaf(__uint_as_float(rs[c1]), sl2, -lv[2 * h + 1]));
-          const float da = __uint_as_float(rp[c0]) - dv[2 * h];
-          const float db = __uint_as_float(rp[c1]) - dv[2 * h + 1];
+          float xa, xb, qa, qb;
+          f2_split(fma2(f2(__uint_as_float(rs[c0]), __uint_as_float(rs[c1])), sl2x2, nl2[h]), xa, xb);
+          const float pa = ex2(xa), pb = ex2(xb);
+          f2_split(mul2(f2(pa, pb), sub2(f2(__uint_as_float(rp[c0]), __uint_as_float(rp[c1])), dv2[h])), qa, qb);
           pk[i] = pack_bf16(pa, pb);
-          dk[i] = pack_bf16(pa * da, pb * db);
+          dk[i] = pack_bf16(qa, qb);
         }
       }
       tmem_st_cols(cS, pk);

@@ -491,12 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           rt[i] = v ? rt[i] : 0u;
         }
       }
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
-      const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float hmax = max_of32(s);
       // Exchange the half-row max with the other warpgroup.
       xch[(b * 2 + g) * BM + row] = hmax;
       if (!pair_sync(bar.pair + 8 * (sub * 2 + b), (j >> 1) & 1, lane, abort_flag, p.timeout_ns,
@@ -540,23 +535,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float ref = (m_run == -INFINITY) ? 0.f : m_run;
       // P = 2^(s*scale*log2e - ref) and P o tS, rounded to bf16 and packed into
       // this half's first 16 score columns.
-      float ls[4] = {0.f, 0.f, 0.f, 0.f}, rsum[4] = {0.f, 0.f, 0.f, 0.f};
+      // Element pairs go through packed fp32x2 arithmetic (the exponentials
+      // stay scalar): the same roundings per element, half the instructions.
+      const uint64_t sl2x2 = f2(sl2, sl2), nref2 = f2(-ref, -ref), scale2 = f2(scale, scale);
+      uint64_t ls2[2] = {0ull, 0ull}, rs2[2] = {0ull, 0ull};
       uint32_t pk[16], tk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-        const float qa = pa * (__uint_as_float(rt[2 * i]) * scale);
-        const float qb = pb * (__uint_as_float(rt[2 * i + 1]) * scale);
-        ls[i & 3] += pa + pb;
-        rsum[i & 3] += qa + qb;
+        float xa, xb;
+        f2_split(fma2(f2(s[2 * i], s[2 * i + 1]), sl2x2, nref2), xa, xb);
+        const float pa = ex2(xa), pb = ex2(xb);
+        const uint64_t p2 = f2(pa, pb);
+        const uint64_t q2 = mul2(p2, mul2(f2(__uint_as_float(rt[2 * i]), __uint_as_float(rt[2 * i + 1])), scale2));
+        ls2[i & 1] = add2(ls2[i & 1], p2);
+        rs2[i & 1] = add2(rs2[i & 1], q2);
+        float qa, qb;
+        f2_split(q2, qa, qb);
         pk[i] = pack_bf16(pa, pb);
         tk[i] = pack_bf16(qa, qb);
       }
       tmem_st16(cS, pk);
       tmem_st16(cT, tk);
-      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      r_run += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+      float la, lb, lc, ld, ra, rb, rc, rd;
+      f2_split(ls2[0], la, lb);
+      f2_split(ls2[1], lc, ld);
+      f2_split(rs2[0], ra, rb);
+      f2_split(rs2[1], rc, rd);
+      l_run += (la + lb) + (lc + ld);
+      r_run += (ra + rb) + (rc + rd);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -897,14 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           s[32 + i] = ((v1 >> i) & 1u) ? s[32 + i] : -INFINITY;
         }
       }
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        mx[i] = fmaxf(fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24])),
-                      fmaxf(fmaxf(s[i + 32], s[i + 40]), fmaxf(s[i + 48], s[i + 56])));
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], mx[i + 4]);
-      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      const float m_tile = fmaxf(max_of32(s), max_of32(s + 32)) * sl2;
       const bool grow = m_tile > m_run + kRescaleThreshold;
       const bool had_acc = m_run != -INFINITY;
       float alpha = 1.f;
@@ -934,21 +933,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float ref = (m_run == -INFINITY) ? 0.f : m_run;
       // P = 2^(s*scale*log2e - ref) in bf16: keys 0-31 packed into columns
       // 0-15, keys 32-63 into columns 32-47 (the layout the value MMA reads)
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // element pairs in packed fp32x2 arithmetic (exponentials scalar)
+      const uint64_t sl2x2 = f2(sl2, sl2), nref2 = f2(-ref, -ref);
+      uint64_t ls2[2] = {0ull, 0ull};
       uint32_t pk0[16], pk1[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float pa = ex2(fmaf(s[2 * i], sl2, -ref));
-        const float pb = ex2(fmaf(s[2 * i + 1], sl2, -ref));
-        const float pc = ex2(fmaf(s[32 + 2 * i], sl2, -ref));
-        const float pd = ex2(fmaf(s[32 + 2 * i + 1], sl2, -ref));
-        ls[i & 3] += (pa + pb) + (pc + pd);
+        float xa, xb, xc, xd;
+        f2_split(fma2(f2(s[2 * i], s[2 * i + 1]), sl2x2, nref2), xa, xb);
+        f2_split(fma2(f2(s[32 + 2 * i], s[32 + 2 * i + 1]), sl2x2, nref2), xc, xd);
+        const float pa = ex2(xa), pb = ex2(xb), pc = ex2(xc), pd = ex2(xd);
+        ls2[i & 1] = add2(ls2[i & 1], add2(f2(pa, pb), f2(pc, pd)));
         pk0[i] = pack_bf16(pa, pb);
         pk1[i] = pack_bf16(pc, pd);
       }
       tmem_st16(cS, pk0);
       tmem_st16(cS + 32, pk1);
-      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      float la, lb, lc, ld;
+      f2_split(ls2[0], la, lb);
+      f2_split(ls2[1], lc, ld);
+      l_run += (la + lb) + (lc + ld);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
