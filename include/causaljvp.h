@@ -229,8 +229,9 @@ caj_status caj_signal_barrier(uint32_t *const *pads, int32_t shards, int32_t ran
  *   caj_ipc_open    maps a handle exported by ANOTHER process (same node) and
  *                   returns the address of the exported ptr in this process;
  *                   peer access is enabled on first touch.
- *   caj_ipc_close   unmaps an address returned by caj_ipc_open. The exporter
- *                   keeps its memory until every opener has closed it.
+ *   caj_ipc_close   unmaps an address returned by caj_ipc_open. An address
+ *                   opened n times needs n closes. The exporter keeps its
+ *                   memory until every opener has closed it.
  * Return CAJ_OK, CAJ_ERR_INVALID_ARG (null argument; an address not opened
  * here) or CAJ_ERR_CUDA (caj_last_cuda_error names the CUDA error).
  */

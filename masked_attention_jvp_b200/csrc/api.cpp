@@ -14,6 +14,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <utility>
 #include <memory>
 #include <mutex>
 #include <vector>
@@ -764,9 +765,11 @@ AddressRangeFn get_address_range() {
   return fn;
 }
 
-// Addresses handed out by caj_ipc_open, with the mapped allocation's base.
+// Addresses handed out by caj_ipc_open, with the mapped allocation's base and
+// how many opens are outstanding (opening a handle that is already mapped in
+// this context returns the same mapping, reference-counted by the runtime).
 std::mutex g_ipc_mu;
-std::map<uintptr_t, void *> g_ipc_open;
+std::map<uintptr_t, std::pair<void *, int>> g_ipc_open;
 }  // namespace
 
 caj_status caj_ipc_export(const void *ptr, caj_ipc_handle *out) {
@@ -794,7 +797,9 @@ caj_status caj_ipc_open(const caj_ipc_handle *h, void **ptr) {
   if (e != cudaSuccess) return cuda_fail(e);
   void *p = static_cast<uint8_t *>(base) + h->offset;
   std::lock_guard<std::mutex> lock(g_ipc_mu);
-  g_ipc_open[reinterpret_cast<uintptr_t>(p)] = base;
+  auto &entry = g_ipc_open[reinterpret_cast<uintptr_t>(p)];
+  entry.first = base;
+  entry.second += 1;
   *ptr = p;
   return CAJ_OK;
 }
@@ -805,8 +810,8 @@ caj_status caj_ipc_close(void *ptr) {
     std::lock_guard<std::mutex> lock(g_ipc_mu);
     auto it = g_ipc_open.find(reinterpret_cast<uintptr_t>(ptr));
     if (!ptr || it == g_ipc_open.end()) return CAJ_ERR_INVALID_ARG;
-    base = it->second;
-    g_ipc_open.erase(it);
+    base = it->second.first;
+    if (--it->second.second == 0) g_ipc_open.erase(it);
   }
   cudaError_t e = cudaIpcCloseMemHandle(base);
   return e == cudaSuccess ? CAJ_OK : cuda_fail(e);

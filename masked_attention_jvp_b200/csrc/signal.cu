@@ -47,8 +47,9 @@ __global__ void signal_barrier_kernel(SignalParams p) {
     store_release_sys(p.pads[t] + p.rank, p.epoch);
     const uint32_t *mine = p.pads[p.rank] + t;
     const uint64_t start = now_ns();
-    while (int32_t(load_acquire_sys(mine) - p.epoch) < 0) {
-      if (now_ns() - start > p.timeout_ns) {
+    // bounded by time and, should the timer misbehave, by a poll count as well
+    for (uint32_t it = 0; int32_t(load_acquire_sys(mine) - p.epoch) < 0; ++it) {
+      if (now_ns() - start > p.timeout_ns || it >= (1u << 30)) {
         atomicCAS(&g_signal_error, 0u, uint32_t(kErrTimeoutBase | kSiteSignalBarrier));
         break;
       }

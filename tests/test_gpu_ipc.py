@@ -35,6 +35,13 @@ def _writer(handles, q):
         mine = [torch.full((B, H, Ls, D), float("nan"), dtype=W.dtype, device="cuda") for _ in range(2)]
         mine += [torch.full((B, H, Ls), float("nan"), device="cuda") for _ in range(2)]
         addrs = [caj2.ipc_open(h) for h in handles]
+        # a second open of a mapped handle gives the same address and needs its
+        # own close; the first mapping stays usable (the scatter below writes
+        # through it)
+        again = caj2.ipc_open(handles[0])
+        if again != addrs[0]:
+            raise AssertionError(f"second open gave {again:#x}, first {addrs[0]:#x}")
+        caj2.ipc_close(again)
         shapes = [((B, H, Ls, D), W.dtype)] * 2 + [((B, H, Ls), torch.float32)] * 2
         peer = [PeerView(a, s, dt) for a, (s, dt) in zip(addrs, shapes)]
         caj2.attn_fwd_jvp_scatter(*ins, W.mask, [mine[0], peer[0]], [mine[1], peer[1]],
