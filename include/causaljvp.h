@@ -248,7 +248,9 @@ caj_status caj_ipc_close(void *ptr);
  * and outputs in host memory. The heads are split into at most 16 chunks.
  * Three things run at once on three streams: the copy of chunk c's six inputs
  * to the device, the kernel on chunk c-1, and the copy of an earlier chunk's
- * outputs back to the host. Pinned host memory lets the copies overlap;
+ * outputs back to the host. (bf16: the first and the last chunk go in two
+ * pieces by query rows, the first piece copying only the key rows its query
+ * tiles read, so the pipeline fills and drains in half the time.) Pinned host memory lets the copies overlap;
  * pageable memory gives the same results, but its copies do not overlap.
  *   in : q, k, v, tq, tk, tv   host, [B,H,N,D] of prob->dtype, read only
  *   out: o, to                 host, [B,H,N,D] of prob->dtype
