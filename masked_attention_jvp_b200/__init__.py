@@ -3,6 +3,7 @@
 Public API (a thin layer over the C-ABI library libcausaljvp):
 
     o, to, lse, tlse = attn_fwd_jvp(q, k, v, tq, tk, tv, mask, scale=None)
+    o, to, lse, tlse = attention_jvp(q, k, v, tq, tk, tv, mask)  # o differentiable in q, k, v
 
 q..tv are [B, H, N, D] tensors (bf16 for the tensor-core path, fp32 for the
 CUDA-core fp32 path), `mask` a MaskDesc (or a (tokens_per_frame,
@@ -28,7 +29,7 @@ from . import _lib
 from ._lib import CajError, EXPORTED, LIB_PATH
 from .workloads import MaskDesc
 
-__all__ = ["attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "signal_barrier",
+__all__ = ["attention_jvp", "attn_fwd_jvp", "attn_fwd_jvp_out", "attn_fwd_jvp_scatter", "attn_fwd_jvp_host_static", "signal_barrier",
            "ipc_export", "ipc_open", "ipc_close", "part_query_tiles", "attn_bwd", "qk_norm_rope_jvp", "out_proj_jvp", "MaskDesc", "CajError", "visible_pairs",
            "row_key_ranges", "qtile_key_tiles", "device_status", "flops", "EXPORTED", "LIB_PATH",
            "BLOCK_M", "BLOCK_N"]
@@ -37,6 +38,8 @@ BLOCK_M = 128  # query rows per tile of both kernels
 BLOCK_N = 64   # keys per tile of the tensor-core kernel
 
 _DTYPES = {torch.float32: _lib.CAJ_DTYPE_F32, torch.bfloat16: _lib.CAJ_DTYPE_BF16}
+
+from .autograd import attention_jvp  # noqa: E402  (autograd binding: fused forward, backward kernels)
 
 
 def part_query_tiles(mask, part: int, nparts: int):
