@@ -628,45 +628,6 @@ def bench_e2e(args, w, host, fl_job, world, stream, dev, barrier):
             "api": "attn_fwd_jvp on pinned CPU tensors (caj_attn_fwd_jvp_host)"}
 
 
-def bench_e2e_part(args, w, host, fl_job, world, rank, stream, dev, barrier):
-    """The e2e leg of the query-tile split: every step each rank copies the
-    whole inputs from pinned host memory, runs its part through the public
-    API (attn_fwd_jvp_out with part=(rank, world)) and copies the four output
-    buffers back to pinned host memory, all on one stream."""
-    import masked_attention_jvp_b200 as caj
-    pinned = [t.pin_memory() for t in host]
-    dins = [torch.empty_like(t, device=dev) for t in pinned]
-    o, to = torch.empty_like(dins[0]), torch.empty_like(dins[0])
-    lse = torch.empty(dins[0].shape[:3], dtype=torch.float32, device=dev)
-    tlse = torch.empty_like(lse)
-    hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, to, lse, tlse)]
-    h2d = sum(t.numel() * t.element_size() for t in pinned)
-    d2h = sum(t.numel() * t.element_size() for t in hout)
-
-    def step():
-        for d, h in zip(dins, pinned):
-            d.copy_(h, non_blocking=True)
-        caj.attn_fwd_jvp_out(*dins, w.mask, o, to, lse, tlse, scale=w.scale, stream=stream, part=(rank, world))
-        for h, d in zip(hout, (o, to, lse, tlse)):
-            h.copy_(d, non_blocking=True)
-
-    step()
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    return {"value": round(strong_tflops(fl_job, args.steps, ms), 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.steps,
-            "ms_per_step": round(ms / args.steps, 3), "clocks": clk.summary(),
-            "api": "attn_fwd_jvp_out(part=(rank, world)) between pinned-host copies, per rank"}
-
-
 def rank_inputs(args, w, host, world, rank):
     """This rank's share of the workload's inputs (host tensors) and the
     problem it runs, by the split mode."""
@@ -751,7 +712,12 @@ def bench_gpu(args, rank, world, local_rank):
     if not args.no_e2e and (world == 1 or args.split in ("heads", "replicas")):
         e2e = bench_e2e(args, w, host, fl_job, world, stream, dev, barrier)
     elif not args.no_e2e and args.split == "tiles":
-        e2e = bench_e2e_part(args, w, host, fl_job, world, rank, stream, dev, barrier)
+        # host-resident inputs: a query-tile share would read every head's keys, so
+        # each rank takes its share of the heads through the pipelined host call
+        h0, h1 = split_heads(w.H, world, rank)
+        share = [t[:, h0:h1].contiguous() for t in host]
+        e2e = bench_e2e(args, w, share, fl_job, world, stream, dev, barrier)
+        e2e["api"] += "; rank r its heads split_heads(H, world, r)"
     if rank != 0:
         return None
     peaks, src = load_peaks()
