@@ -92,6 +92,14 @@ __device__ __forceinline__ bool bwarp_wait(uint32_t bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, bwait(bar, parity, abort_flag, timeout_ns, site));
 }
 
+// Bounded wait of the MMA warp, with no warp vote (see the forward kernels: a
+// vote after queued tensor-core instructions holds the warp until the queue
+// takes them); the warp reconverges after its loop.
+__device__ __forceinline__ bool bissuer_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                             uint64_t timeout_ns, uint32_t site) {
+  return bwait(bar, parity, abort_flag, timeout_ns, site);
+}
+
 __device__ __forceinline__ void bdrain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return;
   const uint64_t t0 = globaltimer_ns();
@@ -298,12 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_ST, 16, 1024);
     const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_ST + C::S_BYTES, 16, 1024);
     const uint64_t dKmn0 = sdesc_sw128(sbase + C::OFF_ST, C::SBLK, 1024);
-    bool ok = bwarp_wait(bar.a_ready, 0, abort_flag, p.timeout_ns, 22);
+    bool ok = bissuer_wait(bar.a_ready, 0, abort_flag, p.timeout_ns, 22);
     tc_fence_after();
     for (int32_t j = 0; ok && j <= ntiles; ++j) {
       if (j < ntiles) {
         const int s = j % C::STAGES;
-        if (!(ok = bwarp_wait(bar.st_full + 8 * s, (j / C::STAGES) & 1, abort_flag, p.timeout_ns, 23)))
+        if (!(ok = bissuer_wait(bar.st_full + 8 * s, (j / C::STAGES) & 1, abort_flag, p.timeout_ns, 23)))
           break;
         const uint64_t so = uint64_t((s * C::STAGE) >> 4);
         const uint32_t cS = tmem + COL_S0 + (j & 1) * 128;
@@ -317,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       }
       if (j >= 1) {
         const int32_t i = j - 1;
-        if (!(ok = bwarp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 24)))
+        if (!(ok = bissuer_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 24)))
           break;
         tc_fence_after();
         const int s = i % C::STAGES;
@@ -333,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
         tc_commit(leader, bar.st_empty + 8 * s);
       }
     }
+    __syncwarp();  // lanes may leave the loop apart on an abort
     tc_commit(leader, bar.drain);
     bdrain(bar.drain, 0, p.timeout_ns);
   } else {
@@ -510,13 +519,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     const uint64_t dO0 = sdesc_sw128(sbase + C::OFF_ST + C::S_BYTES, 16, 1024);
     const uint64_t dQmn0 = sdesc_sw128(sbase + C::OFF_ST, C::SBLK, 1024);
     const uint64_t dOmn0 = sdesc_sw128(sbase + C::OFF_ST + C::S_BYTES, C::SBLK, 1024);
-    bool ok = bwarp_wait(bar.a_ready, 0, abort_flag, p.timeout_ns, 38) &&
-              bwarp_wait(bar.r_full, 0, abort_flag, p.timeout_ns, 32);
+    bool ok = bissuer_wait(bar.a_ready, 0, abort_flag, p.timeout_ns, 38) &&
+              bissuer_wait(bar.r_full, 0, abort_flag, p.timeout_ns, 32);
     tc_fence_after();
     for (int32_t j = 0; ok && j <= ntiles; ++j) {
       if (j < ntiles) {
         const int s = j % C::STAGES;
-        if (!(ok = bwarp_wait(bar.st_full + 8 * s, (j / C::STAGES) & 1, abort_flag, p.timeout_ns, 33)))
+        if (!(ok = bissuer_wait(bar.st_full + 8 * s, (j / C::STAGES) & 1, abort_flag, p.timeout_ns, 33)))
           break;
         const uint64_t so = uint64_t((s * C::STAGE) >> 4);
         const uint32_t cS = tmem + COL_S0 + (j & 1) * 64;
@@ -527,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         }
         // dP^T has one buffer: the softmax must have read dP^T(j-1)
         if (j >= 1) {
-          if (!(ok = bwarp_wait(bar.dp_free, (j - 1) & 1, abort_flag, p.timeout_ns, 39))) break;
+          if (!(ok = bissuer_wait(bar.dp_free, (j - 1) & 1, abort_flag, p.timeout_ns, 39))) break;
           tc_fence_after();
         }
 #pragma unroll
@@ -540,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       }
       if (j >= 1) {
         const int32_t i = j - 1;
-        if (!(ok = bwarp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 34)))
+        if (!(ok = bissuer_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 34)))
           break;
         tc_fence_after();
         const int s = i % C::STAGES;
@@ -560,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         tc_commit(leader, bar.st_empty + 8 * s);
       }
     }
+    __syncwarp();  // lanes may leave the loop apart on an abort
     tc_commit(leader, bar.drain);
     bdrain(bar.drain, 0, p.timeout_ns);
   } else {

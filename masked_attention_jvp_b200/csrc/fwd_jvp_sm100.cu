@@ -194,6 +194,17 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, timeout_ns, site));
 }
 
+// Bounded wait of the MMA warp, with no warp vote: a vote right after the
+// elected lane has queued tensor-core instructions holds the whole warp until
+// the queue takes them (about 390 cycles with a full queue). Every lane polls
+// the same barrier, so the lanes agree but for an abort or a timeout, where a
+// lane that gives up raises the CTA's abort flag and the others follow at
+// their next wait; the warp reconverges after its loop.
+__device__ __forceinline__ bool issuer_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                            uint64_t timeout_ns, uint32_t site) {
+  return wait_bounded(bar, parity, abort_flag, timeout_ns, site);
+}
+
 // The slice-map arithmetic of the scattering epilogues, kept out of line.
 // Inlined, it changed the register allocation of the kernels' main loop:
 // the scattering kernel then ran 4.7% slower than the plain one, against
@@ -367,12 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // MN-major B: 64-element column blocks C::VBLK apart, 8-key groups 1 KiB apart.
     const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::VBLK, 1024);
     const uint32_t tS0 = tmem + C::COL_S0;
-    bool ok = warp_wait(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
+    bool ok = issuer_wait(bar.q_full, 0, abort_flag, p.timeout_ns, 3);
     // Step j: scores of key tile j, then value products of key tile j-1. One
     // probe covers K(j) and V(j-1), a second one P(j-1). A probe issued while
     // earlier MMAs are still queued overlaps their execution, so each probe is
     // placed kProbeLead k-steps before the end of the batch that precedes its use.
-    if (ok) ok = warp_wait(bar.x_full, 0, abort_flag, p.timeout_ns, 4);
+    if (ok) ok = issuer_wait(bar.x_full, 0, abort_flag, p.timeout_ns, 4);
     for (int32_t j = 0; ok && j <= ntiles; ++j) {
       const int32_t i = j - 1;  // key tile whose value products this step issues
       bool have_p = i < 0;
@@ -383,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           if (kk == D / 16 - kProbeLeadS && !have_p) {
-            if (!(ok = warp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
+            if (!(ok = issuer_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
               break;
             have_p = true;
           }
@@ -405,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool have_x = !next;
       if (i >= 0) {
         if (!have_p &&
-            !(ok = warp_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
+            !(ok = issuer_wait(bar.p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag, p.timeout_ns, 5)))
           break;
         tc_fence_after();
         const uint64_t dV = dV0 + uint64_t(((i & 1) * C::V_STAGE) >> 4);
@@ -415,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           if (kk == BN / 16 - kProbeLeadV && !have_x) {
-            if (!(ok = warp_wait(bar.x_full + 8 * ((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag,
+            if (!(ok = issuer_wait(bar.x_full + 8 * ((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag,
                                  p.timeout_ns, 4)))
               break;
             have_x = true;
@@ -434,11 +445,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(leader, bar.o_done + 8 * (i & 1));
       }
       if (!have_x &&
-          !(ok = warp_wait(bar.x_full + 8 * ((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag,
+          !(ok = issuer_wait(bar.x_full + 8 * ((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag,
                            p.timeout_ns, 4)))
         break;
     }
     // Drain: all MMAs issued by the elected lane complete before TMEM is freed.
+    __syncwarp();  // lanes may leave the loop apart on an abort
     tc_commit(leader, bar.drain);
     drain_wait(bar.drain, 0, p.timeout_ns);
   } else {
@@ -817,13 +829,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
     const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
     const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::KBLK, 1024);
-    bool ok = warp_wait(bar.q_full, 0, abort_flag, p.timeout_ns, 14);
+    bool ok = issuer_wait(bar.q_full, 0, abort_flag, p.timeout_ns, 14);
     for (int32_t j = 0; ok && j < ntiles + kPrimalLag; ++j) {
       if (j < ntiles) {
         // Buffer j%NS last held P of tile j - NS, read by its value product,
         // which was issued earlier (step j - 1): the tensor pipe runs in order.
         const int b = j % NS;
-        if (!(ok = warp_wait(bar.k_full + 8 * b, (j / NS) & 1, abort_flag, p.timeout_ns, 15))) break;
+        if (!(ok = issuer_wait(bar.k_full + 8 * b, (j / NS) & 1, abort_flag, p.timeout_ns, 15))) break;
         tc_fence_after();
         const uint64_t dK = dK0 + uint64_t((b * C::K_STAGE) >> 4);
         const uint32_t dS = tmem + C::COL_S0 + b * BN;
@@ -838,8 +850,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t i = j - kPrimalLag;
       if (i >= 0) {
         const int b = i % NS;
-        if (!(ok = warp_wait(bar.p_full + 8 * b, (i / NS) & 1, abort_flag, p.timeout_ns, 16))) break;
-        if (!(ok = warp_wait(bar.v_full + 8 * b, (i / NS) & 1, abort_flag, p.timeout_ns, 17))) break;
+        if (!(ok = issuer_wait(bar.p_full + 8 * b, (i / NS) & 1, abort_flag, p.timeout_ns, 16))) break;
+        if (!(ok = issuer_wait(bar.v_full + 8 * b, (i / NS) & 1, abort_flag, p.timeout_ns, 17))) break;
         tc_fence_after();
         const uint64_t dV = dV0 + uint64_t((b * C::V_STAGE) >> 4);
         const uint32_t aP = tmem + C::COL_S0 + b * BN;
@@ -853,6 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(leader, bar.o_done + 8 * b);
       }
     }
+    __syncwarp();  // lanes may leave the loop apart on an abort
     tc_commit(leader, bar.drain);
     drain_wait(bar.drain, 0, p.timeout_ns);
   } else {
